@@ -1,0 +1,485 @@
+"""Benchmark of the theta-bundle linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gemma3_decode|gemma3_g1|gemma4_decode|gemma4_prefill]
+
+One step = one pass of the hot path over one batch of synthetic input.  The
+default workload is the Gemma-3-1B-shaped decode: 26 layers in 13 bands
+(G = 13), rank 16, M = 1 token, every layer's q/k/v (stacked), o, gate/up
+(stacked) and down projections.  The metric is weight GB/s: unique parameter
+bytes a step must stream (each band's W0 once, every layer's s, U, V) divided
+by the step time.  Inputs are resident in HBM before timing; per step they
+total more than 3x the 126 MB L2.
+
+Timed region: CUDA-graph replays of the whole step (W >= 3 warm-up steps, then
+exactly K steps between two barrier + synchronize pairs, CUDA events on the
+launching stream, max over ranks).  The JSON line adds:
+  e2e          the same metric through the public Python API, eager, with the
+               step's x copied host->device from pinned memory and all y copied
+               back every step;
+  roofline     for the dominant kernel (the gate/up stacked decode call),
+               timed alone over rotating buffers;
+  cpu_baseline the fp64 oracle on the host, on a bounded sample of the step;
+  secondary    the other workloads' headline figures (Gemma-4-31B decode
+               GB/s, Gemma-4-31B prefill TFLOP/s).
+With --gpus N > 1 each rank runs an independent replica (the path has no
+exchange step); value is the total over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import wl_inputs  # noqa: E402
+from linear_wl_forward_b200 import footprint  # noqa: E402
+
+METRIC = "decode weight GB/s (% of HBM peak); prefill TFLOP/s (% bf16 TC peak)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ utils --
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.out is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.out.flush()
+        with open(self.out.name) as f:
+            rows = [[c.strip() for c in line.split(",")] for line in f if line.count(",") >= 8]
+        os.unlink(self.out.name)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def to_dev_call(call):
+    return {"x": call.x.cuda(),
+            "projs": [(p.W0.cuda(), p.s.cuda(), p.U.cuda() if p.r else None,
+                       p.V.cuda() if p.r else None) for p in call.projs]}
+
+
+def launches_per_call(call, path):
+    """Kernels one call launches (the library's own kernels)."""
+    rs = [p.r for p in call.projs]
+    if path == "decode":
+        return 1 + (1 if any(rs) else 0)
+    n = 1
+    if any(rs):
+        n += sum(1 for r in rs if r) + 1  # V transposes + the T = x V GEMM
+        n += sum(1 for r in rs if r and r % 8)  # padded U copies
+    return n
+
+
+def call_path(call):
+    return "decode" if call.x.shape[0] <= 4 else "gemm"
+
+
+# ------------------------------------------------------------- workloads --
+def build_workload(name):
+    """Returns (calls, unique_weight_bytes, flops, description)."""
+    if name == "gemma3_decode":
+        calls = wl_inputs.gemma3_sweep(seed=2, G=13, r=16, M=1)
+        desc = {"workload": "Gemma-3-1B-shaped decode sweep", "layers": 26, "bands_G": 13,
+                "rank": 16, "M": 1, "hidden": 1152}
+    elif name == "gemma3_g1":
+        calls = wl_inputs.gemma3_sweep(seed=3, G=1, r=64, M=8)
+        desc = {"workload": "Gemma-3-1B-shaped stacked decode, G=1", "layers": 26, "rank": 64,
+                "M": 8}
+    elif name == "gemma4_decode":
+        calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=range(12))
+        desc = {"workload": "Gemma-4-31B-shaped decode, band 0 (layers 0-11)", "rank": 256,
+                "M": 1, "hidden": 5376}
+    elif name == "gemma4_prefill":
+        calls = wl_inputs.gemma4_calls(seed=5, r=256, M=4096, layers=[0])
+        desc = {"workload": "Gemma-4-31B-shaped prefill, sliding layer 0", "rank": 256,
+                "M": 4096, "hidden": 5376}
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    seen = set()
+    wbytes = 0
+    flops = 0
+    for c in calls:
+        M = c.x.shape[0]
+        for p in c.projs:
+            if id(p.W0) not in seen:
+                seen.add(id(p.W0))
+                wbytes += p.N * p.K * 2
+            wbytes += (p.N + p.K) * p.r * 2 + p.N * 4
+            flops += footprint.call_flops(M, p.N, p.K, p.r)
+    return calls, wbytes, flops, desc
+
+
+def make_step(dev_calls, outs, wl):
+    def step():
+        for dc, ys in zip(dev_calls, outs):
+            wl.stacked_forward(dc["x"], dc["projs"], ys=ys)
+    return step
+
+
+def alloc_outputs(calls, out_flat=None):
+    outs = []
+    off = 0
+    for c in calls:
+        M = c.x.shape[0]
+        ys = []
+        for p in c.projs:
+            n = M * p.N
+            if out_flat is not None:
+                ys.append(out_flat[off:off + n].view(M, p.N))
+            else:
+                ys.append(torch.empty(M, p.N, dtype=torch.bfloat16, device="cuda"))
+            off += n
+        outs.append(ys)
+    return outs, off
+
+
+def capture(step, warmup):
+    for _ in range(max(warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, reps):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(reps):
+        g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / reps  # ms
+
+
+# --------------------------------------------------------------- roofline --
+def decode_roofline(wl, peaks):
+    """Dominant kernel of the Gemma-3-1B decode step: the stacked gate/up
+    decode call (2 x 4096 x 1152, rank 16, M = 1).  Timed alone with CUDA
+    events over a graph of calls that rotate through enough distinct bundles
+    (> 3x L2) that every launch streams its weights from HBM."""
+    N, K, r, M = 4096, 1152, 16, 1
+    per_call = 2 * footprint.call_weight_bytes(N, K, r) + footprint.call_io_bytes(M, 2 * N, K)
+    copies = max(4, (3 * L2_BYTES) // (2 * N * K * 2) + 1)
+    calls = []
+    for i in range(copies):
+        c = wl_inputs.random_case(1000 + i, M, [N, N], K, [r, r], P=2)
+        calls.append(to_dev_call(c))
+    outs = [[torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+            for _ in calls]
+    step = make_step(calls, outs, wl)
+    g = capture(step, 3)
+    ms = time_graph(g, 20) / copies
+    achieved = per_call / (ms * 1e-3) / 1e9
+    traffic = traffic_from_profile("decode_kernel")
+    return {"kernel": "decode_kernel<1> (+ tvec_kernel<1>, PDL-overlapped)",
+            "call": "stacked gate/up decode, 2 x 4096 x 1152, r=16, M=1",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "algorithmic_bytes": per_call, "us_per_launch": round(ms * 1e3, 3),
+            "peak_source": peaks["source"]}
+
+
+def traffic_from_profile(kernel):
+    """DRAM bytes per launch from the committed ncu summary, only while the
+    kernel source is unchanged since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "linear_wl_forward_b200", "csrc", rec["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if h == rec["source_sha"] else None
+
+
+# -------------------------------------------------------------- secondary --
+def secondary_figures(wl, peaks):
+    out = {}
+    # Gemma-4-31B decode, M = 1: stacked gate/up of two bands (rotating, > L2)
+    calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=[0, 12], families=("gate",))
+    dev = [to_dev_call(c) for c in calls]
+    outs, _ = alloc_outputs(calls)
+    g = capture(make_step(dev, outs, wl), 3)
+    ms = time_graph(g, 10) / len(calls)
+    p0 = calls[0].projs
+    b = sum(footprint.call_weight_bytes(p.N, p.K, p.r) for p in p0)
+    out["gemma4_decode_gate_up_M1"] = {
+        "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "us_per_call": round(ms * 1e3, 2), "weight_bytes_per_call": b}
+    del dev, outs, g
+    torch.cuda.empty_cache()
+    # Gemma-4-31B prefill, M = 4096: stacked gate/up of layer 0
+    calls = wl_inputs.gemma4_calls(seed=5, r=256, M=4096, layers=[0], families=("gate",))
+    dev = [to_dev_call(c) for c in calls]
+    outs, _ = alloc_outputs(calls)
+    g = capture(make_step(dev, outs, wl), 3)
+    ms = time_graph(g, 5)
+    c = calls[0]
+    fl = sum(footprint.call_flops(4096, p.N, p.K, p.r) for p in c.projs)
+    tf = fl / (ms * 1e-3) / 1e12
+    out["gemma4_prefill_gate_up_M4096"] = {
+        "TFLOP/s": round(tf, 1), "tc_frac": round(tf / peaks["bf16_tflops"], 4),
+        "ms_per_call": round(ms, 3), "flops_per_call": fl, "peak": peaks["bf16_tflops"]}
+    return out
+
+
+# ---------------------------------------------------------- CPU baseline --
+def oracle_sample(calls, budget_s=12.0):
+    """The fp64 oracle on the host over whole calls of the step until the
+    time budget is spent; returns (weight bytes processed, seconds, calls)."""
+    import oracle
+
+    t0 = time.perf_counter()
+    done_b = 0
+    n = 0
+    seen = set()
+    for c in calls:
+        for p in c.projs:
+            oracle.forward(c.x, p.W0, p.s, p.U, p.V)
+            if id(p.W0) not in seen:
+                seen.add(id(p.W0))
+                done_b += p.N * p.K * 2
+            done_b += (p.N + p.K) * p.r * 2 + p.N * 4
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return done_b, time.perf_counter() - t0, n
+
+
+# ------------------------------------------------------------------- main --
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    calls, wbytes, _, desc = build_workload(args.workload)
+    for _ in range(args.warmup):
+        oracle_sample(calls[:4], budget_s=0.5)
+    samples = []
+    for _ in range(args.steps):
+        b, s, n = oracle_sample(calls, budget_s=max(2.0, 60.0 / max(args.steps, 1)))
+        samples.append((b, s, n))
+    b = sum(x[0] for x in samples)
+    s = sum(x[1] for x in samples)
+    v = b / s / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(s / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(desc, sample="oracle over whole calls of the step, bounded by time"),
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{sum(x[2] for x in samples)} calls over {args.steps} steps"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gemma3_decode")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import linear_wl_forward_b200 as wl
+
+    wl.lib()  # fails loudly if the CUDA library is missing
+    peaks = load_peaks()
+
+    calls, wbytes, flops, desc = build_workload(args.workload)
+    dev_calls = [to_dev_call(c) for c in calls]
+    total_out = sum(c.x.shape[0] * p.N for c in calls for p in c.projs)
+    out_flat = torch.empty(total_out, dtype=torch.bfloat16, device="cuda")
+    outs, _ = alloc_outputs(calls, out_flat)
+    step = make_step(dev_calls, outs, wl)
+    launches = sum(launches_per_call(c, call_path(c)) for c in calls)
+
+    graph = capture(step, args.warmup)
+    for _ in range(args.warmup):
+        graph.replay()
+    assert wl.last_device_status() == 0
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for _ in range(args.steps):
+            graph.replay()
+        end.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms_total], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    status = wl.last_device_status()
+    ms_step = ms_total / args.steps
+    value = world * wbytes * args.steps / (ms_total * 1e-3) / 1e9
+
+    # e2e: eager public API calls, x H2D from pinned memory, all y D2H, per step
+    xs_host = {}
+    for c in calls:
+        key = id(c.x)
+        if key not in xs_host:
+            xs_host[key] = c.x.pin_memory()
+    x_dev = {k: next(dc["x"] for c, dc in zip(calls, dev_calls) if id(c.x) == k) for k in xs_host}
+    y_host = torch.empty(total_out, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * 2 for t in xs_host.values())
+    d2h = total_out * 2
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        for k, t in xs_host.items():
+            x_dev[k].copy_(t, non_blocking=True)
+        step()
+        y_host.copy_(out_flat, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(2):
+        e2e_step()
+    if world > 1:
+        torch.distributed.barrier()
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * wbytes / (e2e_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) bf16 bundles, U(0.9,1.1) fp32 s, N(0,1) bf16 x)",
+        "config": dict(desc, parallelism=f"replicas{world}" if world > 1 else "single GPU",
+                       unique_weight_bytes_per_step=wbytes,
+                       l2="inputs larger than L2: each step streams %.0f MB of unique weights"
+                          % (wbytes / 1e6),
+                       timing="CUDA graph of the whole step, replayed K times"),
+        "hbm_frac": round(value / world / peaks["hbm_gbs"], 4),
+        "peaks": peaks,
+        "gpu_launches": launches * args.steps,
+        "device_status": wl.STATUS.get(status, status),
+        "clocks": clk.summary(),
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+                "how": "eager Python API calls per projection stack, x H2D (pinned) and all y D2H"},
+    }
+    if rank == 0 and world == 1:
+        line["roofline"] = decode_roofline(wl, peaks)
+        if not args.no_secondary:
+            line["secondary"] = secondary_figures(wl, peaks)
+        b, s, n = oracle_sample(calls, budget_s=12.0)
+        line["cpu_baseline"] = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"first {n} of {len(calls)} calls of one step "
+                                          f"({b / 1e6:.0f} MB of weights, {s:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

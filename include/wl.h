@@ -1,0 +1,170 @@
+/*
+ * wl.h -- C ABI of the B200 theta-bundle linear ("weightless" linear).
+ *
+ * A theta bundle replaces one dense projection weight by a shared block W0, a
+ * per-output-row scale s and a rank-r delta (U, V), and the layer computes
+ *
+ *     y = s (.) (W0 x) + U (V^T x)
+ *
+ * ("Add a new model architecture", introduction: the theta bundle rebuilds one
+ * projection's weight as y = s.(W0 x) + U.(V^T x)).  W0 is shared by all layers
+ * of a band ("Quality": G = shared_blocks sets how many layers share one W0);
+ * s, U, V belong to one layer.
+ *
+ * Conventions for every entry point below
+ * ---------------------------------------
+ *  - Element types: wl_bf16 is a raw IEEE bfloat16 bit pattern; s is float32.
+ *  - Layouts are row-major: x is M x K (one token per row), W0 is N x K (the
+ *    Linear.weight orientation: rows are outputs), U is N x r, V is K x r,
+ *    y is M x N.  In row-major terms the layer computes Y = X W0^T scaled per
+ *    column n by s[n], plus (X V) U^T.
+ *  - Pointers passed to the forward calls are DEVICE pointers on the current
+ *    CUDA device, owned by the caller; the library never frees or retains them
+ *    beyond the call's kernels.
+ *  - Forward calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  They do not synchronise the host.  They need
+ *    scratch on the device (the low-rank product V^T x and, for large M, a
+ *    transposed copy of V); it comes from a library-owned per-device pool that
+ *    grows on first use of a larger size and is then reused, so calls of a
+ *    repeated shape do not allocate.  Calls that overlap on the GPU (different
+ *    streams, or different host threads) share that pool and must not run
+ *    concurrently; calls on one stream are always safe.
+ *  - Accumulation is fp32 (tensor cores or CUDA cores); y is rounded once to
+ *    bf16 (round to nearest even).  No atomics take part in any sum, so results
+ *    are reproducible run to run.
+ *  - Errors are returned, never aborted on: argument problems are detected on
+ *    the host before anything is launched; launch failures give WL_ERR_CUDA; a
+ *    device-side wait that exceeded its time limit is reported later by
+ *    wl_last_device_status().
+ */
+#ifndef WL_H_
+#define WL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t wl_bf16;
+
+typedef enum {
+    WL_OK = 0,
+    WL_ERR_INVALID_ARG = 1, /* null pointer where data is needed, negative size   */
+    WL_ERR_ALIGNMENT = 2,   /* K % 8 != 0, or x / W0 not 16-byte aligned          */
+    WL_ERR_UNSUPPORTED = 3, /* r > WL_MAX_RANK, P > WL_MAX_PROJ, no sm_100 device */
+    WL_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed      */
+    WL_ERR_TIMEOUT = 5,     /* a device-side wait gave up (see wl_last_device_status) */
+    WL_ERR_NOMEM = 6        /* scratch pool could not grow                          */
+} wl_status;
+
+#define WL_MAX_RANK 1024
+#define WL_MAX_PROJ 8
+
+/* One projection of a stacked call ("Quality (Gemma 4 31B)", "Kernel
+ * optimizations", GEMM path item 1: q/k/v -- or gate/up -- share x).
+ * All pointers are device pointers.  U and V may be NULL iff r == 0. */
+typedef struct {
+    const wl_bf16 *W0; /* N x K, row-major, 16-byte aligned            */
+    const float *s;    /* N                                            */
+    const wl_bf16 *U;  /* N x r, row-major                             */
+    const wl_bf16 *V;  /* K x r, row-major                             */
+    wl_bf16 *y;        /* M x N, row-major (output)                    */
+    int N;             /* output rows of this projection, >= 0         */
+    int r;             /* rank of the delta, 0 <= r <= WL_MAX_RANK     */
+} wl_proj;
+
+/* Which kernels a forward call uses.  WL_PATH_AUTO picks by M; the others exist
+ * so tests and benchmarks can exercise each kernel on any shape. */
+typedef enum {
+    WL_PATH_AUTO = 0,
+    WL_PATH_DECODE = 1, /* streaming CUDA-core kernel, 1 <= M <= WL_DECODE_MAX_M */
+    WL_PATH_GEMM = 2    /* tcgen05 tensor-core GEMM with the fused low-rank epilogue */
+} wl_path;
+
+#define WL_DECODE_MAX_M 4
+
+/* y = s (.) (W0 x) + U (V^T x) for one projection of one layer
+ * ("Add a new model architecture", introduction; the delta is never
+ * materialised as U V^T).
+ *   x  : device, M x K bf16 row-major, 16-byte aligned
+ *   W0 : device, N x K bf16 row-major, 16-byte aligned
+ *   s  : device, N fp32
+ *   U  : device, N x r bf16 row-major (NULL iff r == 0)
+ *   V  : device, K x r bf16 row-major (NULL iff r == 0)
+ *   y  : device, M x N bf16 row-major (written)
+ * M, N >= 0 (0 is a no-op), K >= 0 with K % 8 == 0 (K == 0 writes y = 0),
+ * 0 <= r <= WL_MAX_RANK.  Asynchronous on `stream` (cudaStream_t). */
+wl_status wl_linear_forward(const wl_bf16 *x, const wl_bf16 *W0, const float *s,
+                            const wl_bf16 *U, const wl_bf16 *V, wl_bf16 *y,
+                            int M, int N, int K, int r, void *stream);
+
+/* Several projections against one shared x in one pass ("Quality (Gemma 4
+ * 31B)", "Kernel optimizations", GEMM path item 1: one fused W0 + V product and
+ * a block-diagonal U product instead of one call per child).  projs is a HOST
+ * array of P (1 <= P <= WL_MAX_PROJ) descriptors whose pointers are device
+ * pointers; every projection has the same K.  Projection p writes its own
+ * y_p (M x N_p), using only its own s_p, U_p and V_p.  Same conventions and
+ * errors as wl_linear_forward. */
+wl_status wl_stacked_forward(const wl_bf16 *x, int M, int K, const wl_proj *projs,
+                             int P, void *stream);
+
+/* wl_stacked_forward with an explicit kernel choice (see wl_path).
+ * WL_PATH_DECODE requires M <= WL_DECODE_MAX_M (else WL_ERR_UNSUPPORTED). */
+wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                        wl_path path, void *stream);
+
+/* Host-side decomposition of L dense layer weights into theta bundles
+ * ("Quality", "Why sharing fails": band-mean W0, per-row scale s, low-rank
+ * residual; "Add a new model architecture", "Decompose HF weights" step 4).
+ *   W             : host, L x N x K fp32 (layer-major, each N x K row-major)
+ *   band_of_layer : host, L ints in [0, G), or NULL for contiguous equal bands
+ *                   band(l) = floor(l * G / L)
+ *   W0 (out)      : host, G x N x K fp32 -- mean of each band's layers (zero
+ *                   for a band with no layers)
+ *   s  (out)      : host, L x N fp32 -- least-squares per-row scale
+ *                   <W_l[n], W0[n]> / ||W0[n]||^2 (1 where W0[n] = 0)
+ *   U  (out)      : host, L x N x r fp32 -- left singular vectors times
+ *                   singular values of R_l = W_l - diag(s_l) W0
+ *   V  (out)      : host, L x K x r fp32 -- right singular vectors of R_l
+ *                   (columns beyond rank(R_l) are zero)
+ *   rel_err (out) : host, L doubles, may be NULL -- relative Frobenius error
+ *                   of diag(s) W0 + U V^T against W_l, in fp64 from the fp32
+ *                   factors
+ * Computes in fp64 on the calling thread, synchronously.  Returns
+ * WL_ERR_INVALID_ARG for null pointers, L, N, K, G < 1, r < 0 or a band index
+ * outside [0, G); WL_ERR_NOMEM if host memory runs out. */
+wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r,
+                       const int *band_of_layer, float *W0, float *s, float *U,
+                       float *V, double *rel_err);
+
+/* ||W - (diag(s) W0 + U V^T)||_F / ||W||_F for one layer, host pointers, fp64
+ * ("Quality": relative Frobenius error of diag(s).W0 + U.V^T against the true
+ * weight).  Returns a negative value for invalid arguments. */
+double wl_relative_frobenius_error(const float *W, const float *W0, const float *s,
+                                   const float *U, const float *V, int N, int K, int r);
+
+/* Static description of a status code. */
+const char *wl_status_string(wl_status status);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word: WL_OK, or the first error a kernel recorded since the last call (for
+ * example WL_ERR_TIMEOUT from a wait that gave up). */
+wl_status wl_last_device_status(void *stream);
+
+/* Launches one probe kernel that waits on a device flag nothing ever sets,
+ * giving up after `limit_ns` nanoseconds and recording WL_ERR_TIMEOUT in the
+ * device status word, exactly as the forward kernels do when one of their
+ * waits expires.  Lets tests check the time-out path without a hung GPU.
+ * 0 < limit_ns <= 1e9.  Asynchronous on `stream`. */
+wl_status wl_wait_probe(long long limit_ns, void *stream);
+
+/* Library version, (major << 16) | minor. */
+int wl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WL_H_ */

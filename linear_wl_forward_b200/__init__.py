@@ -1,0 +1,181 @@
+"""Python binding of the B200 theta-bundle linear (``libwl.so``, include/wl.h).
+
+Argument marshalling only: torch tensors are checked for dtype, device and
+layout and their pointers are handed to the C ABI; every step of the forward
+runs in the library's CUDA kernels.  There is no fallback: if the library is
+missing or was built for another device, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "WLError", "lib", "linear_forward", "stacked_forward", "decompose",
+    "relative_frobenius_error", "last_device_status", "wait_probe", "PATHS",
+    "DECODE_MAX_M", "MAX_RANK", "MAX_PROJ", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwl.so")
+
+STATUS = {0: "WL_OK", 1: "WL_ERR_INVALID_ARG", 2: "WL_ERR_ALIGNMENT", 3: "WL_ERR_UNSUPPORTED",
+          4: "WL_ERR_CUDA", 5: "WL_ERR_TIMEOUT", 6: "WL_ERR_NOMEM"}
+PATHS = {"auto": 0, "decode": 1, "gemm": 2}
+DECODE_MAX_M = 4
+MAX_RANK = 1024
+MAX_PROJ = 8
+
+
+class WLError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        self.name = STATUS.get(code, str(code))
+        super().__init__(f"{what}: {self.name} ({_lib.wl_status_string(code).decode() if _lib else ''})")
+
+
+class _Proj(ctypes.Structure):
+    _fields_ = [("W0", ctypes.c_void_p), ("s", ctypes.c_void_p), ("U", ctypes.c_void_p),
+                ("V", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int),
+                ("r", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libwl.so (built by ``python -m linear_wl_forward_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m linear_wl_forward_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci, cll = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
+        L.wl_linear_forward.argtypes = [vp] * 6 + [ci] * 4 + [vp]
+        L.wl_stacked_forward.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, vp]
+        L.wl_forward_ex.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, ci, vp]
+        L.wl_decompose.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp]
+        L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
+        L.wl_relative_frobenius_error.restype = ctypes.c_double
+        L.wl_status_string.argtypes = [ci]
+        L.wl_status_string.restype = ctypes.c_char_p
+        L.wl_last_device_status.argtypes = [vp]
+        L.wl_wait_probe.argtypes = [cll, vp]
+        L.wl_version.restype = ci
+        for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose",
+                     "wl_last_device_status", "wl_wait_probe"):
+            getattr(L, name).restype = ci
+        _lib = L
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise WLError(code, what)
+
+
+def _stream_handle(stream):
+    import torch
+
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dev_ptr(t, dtype, name, shape=None):
+    import torch
+
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _make_proj(W0, s, U, V, y, M, K):
+    import torch
+
+    N = W0.shape[0]
+    r = 0 if U is None else U.shape[1]
+    return _Proj(_dev_ptr(W0, torch.bfloat16, "W0", (N, K)), _dev_ptr(s, torch.float32, "s", (N,)),
+                 _dev_ptr(U, torch.bfloat16, "U", (N, r)) if r else None,
+                 _dev_ptr(V, torch.bfloat16, "V", (K, r)) if r else None,
+                 _dev_ptr(y, torch.bfloat16, "y", (M, N)), N, r)
+
+
+def linear_forward(x, W0, s, U, V, y=None, stream=None, path="auto"):
+    """y = s * (W0 x) + U (V^T x).  x: M x K bf16, W0: N x K bf16, s: N fp32,
+    U: N x r bf16, V: K x r bf16 (U = V = None for r = 0).  Returns y (M x N
+    bf16); asynchronous on `stream` (default: torch's current stream)."""
+    return stacked_forward(x, [(W0, s, U, V)], ys=None if y is None else [y], stream=stream,
+                           path=path)[0]
+
+
+def stacked_forward(x, projs, ys=None, stream=None, path="auto"):
+    """Several projections (W0_p, s_p, U_p, V_p) against one shared x in one
+    call.  Returns the list of y_p (M x N_p bf16)."""
+    import torch
+
+    M, K = x.shape
+    if ys is None:
+        ys = [torch.empty(M, W0.shape[0], dtype=torch.bfloat16, device=x.device)
+              for (W0, _, _, _) in projs]
+    arr = (_Proj * len(projs))(*[_make_proj(W0, s, U, V, y, M, K)
+                                 for (W0, s, U, V), y in zip(projs, ys)])
+    xp = _dev_ptr(x, torch.bfloat16, "x", (M, K))
+    _check(lib().wl_forward_ex(xp, M, K, arr, len(projs), PATHS[path], _stream_handle(stream)),
+           "wl_forward_ex")
+    return ys
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status word."""
+    return lib().wl_last_device_status(_stream_handle(stream))
+
+
+def wait_probe(limit_ns: int, stream=None):
+    _check(lib().wl_wait_probe(int(limit_ns), _stream_handle(stream)), "wl_wait_probe")
+
+
+def decompose(W, G: int, r: int, band_of_layer=None):
+    """Host decomposition (include/wl.h, wl_decompose).  W: (L, N, K) float32
+    numpy array.  Returns (W0 (G,N,K), s (L,N), U (L,N,r), V (L,K,r), rel_err (L,))."""
+    import numpy as np
+
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    L, N, K = W.shape
+    W0 = np.empty((G, N, K), np.float32)
+    s = np.empty((L, N), np.float32)
+    U = np.empty((L, N, r), np.float32)
+    V = np.empty((L, K, r), np.float32)
+    err = np.empty(L, np.float64)
+    bands = None
+    if band_of_layer is not None:
+        bands = np.ascontiguousarray(band_of_layer, dtype=np.int32)
+    _check(lib().wl_decompose(W.ctypes.data, L, N, K, G, r,
+                              None if bands is None else bands.ctypes.data, W0.ctypes.data,
+                              s.ctypes.data, U.ctypes.data, V.ctypes.data, err.ctypes.data),
+           "wl_decompose")
+    return W0, s, U, V, err
+
+
+def relative_frobenius_error(W, W0, s, U, V) -> float:
+    import numpy as np
+
+    W, W0, s = (np.ascontiguousarray(a, dtype=np.float32) for a in (W, W0, s))
+    N, K = W.shape
+    r = 0 if U is None else U.shape[1]
+    U = np.ascontiguousarray(U, dtype=np.float32) if r else None
+    V = np.ascontiguousarray(V, dtype=np.float32) if r else None
+    return lib().wl_relative_frobenius_error(W.ctypes.data, W0.ctypes.data, s.ctypes.data,
+                                             None if U is None else U.ctypes.data,
+                                             None if V is None else V.ctypes.data, N, K, r)

@@ -1,0 +1,395 @@
+// C ABI of the theta-bundle linear: argument checks, the per-device scratch
+// pool, tensor-map encoding and kernel selection.  Declarations and the
+// contract of every entry point are in include/wl.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/wl.h"
+#include "wl_internal.h"
+
+namespace wl {
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per device-side wait
+constexpr int kMaxDevices = 64;
+
+enum Slot { kSlotT = 0, kSlotTPart, kSlotVt, kSlotUPad0, kNumSlots = kSlotUPad0 + kMaxSeg };
+
+struct DevicePool {
+    bool ready = false;
+    int num_sms = 0;
+    int major = 0;
+    int *words = nullptr;  // [0] status, [1] probe flag (never set), [8..15] counters
+    void *buf[kNumSlots] = {};
+    size_t cap[kNumSlots] = {};
+};
+
+std::mutex g_mu;
+DevicePool g_pool[kMaxDevices];
+
+wl_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WL_OK : WL_ERR_CUDA; }
+
+wl_status pool_for_current_device(DevicePool **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WL_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return WL_ERR_UNSUPPORTED;
+    DevicePool &p = g_pool[dev];
+    if (!p.ready) {
+        if (cudaDeviceGetAttribute(&p.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&p.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return WL_ERR_CUDA;
+        if (cudaMalloc(&p.words, 64 * sizeof(int)) != cudaSuccess) return WL_ERR_NOMEM;
+        if (cudaMemset(p.words, 0, 64 * sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
+        if (cudaDeviceSynchronize() != cudaSuccess) return WL_ERR_CUDA;
+        p.ready = true;
+    }
+    if (p.major != 10) return WL_ERR_UNSUPPORTED;  // kernels are built for sm_100a only
+    *out = &p;
+    return WL_OK;
+}
+
+// Grow-only scratch.  Growing waits for the device so no kernel still uses
+// the old buffer; steady-state calls of one shape never reach cudaMalloc.
+wl_status scratch(DevicePool &p, int slot, size_t bytes, void **out) {
+    if (bytes == 0) bytes = 16;
+    if (p.cap[slot] < bytes) {
+        size_t want = std::max(bytes, p.cap[slot] * 2);
+        want = (want + (2u << 20) - 1) & ~size_t((2u << 20) - 1);
+        if (p.buf[slot]) {
+            if (cudaDeviceSynchronize() != cudaSuccess) return WL_ERR_CUDA;
+            cudaFree(p.buf[slot]);
+            p.buf[slot] = nullptr;
+            p.cap[slot] = 0;
+        }
+        if (cudaMalloc(&p.buf[slot], want) != cudaSuccess) {
+            cudaGetLastError();
+            return WL_ERR_NOMEM;
+        }
+        p.cap[slot] = want;
+    }
+    *out = p.buf[slot];
+    return WL_OK;
+}
+
+// ------------------------------------------------------------ tensor maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 map: `rows` x `cols` elements, row stride `ld` elements, box
+// box_rows x 64 elements (128 B, swizzled 128 B).  Out-of-range reads give 0.
+wl_status make_map(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
+                   uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return WL_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------- validation --
+// Pure host checks; touches no CUDA API, so it is testable without a GPU.
+wl_status validate(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, wl_path path) {
+    if (!projs) return WL_ERR_INVALID_ARG;
+    if (P < 1 || P > WL_MAX_PROJ) return P < 1 ? WL_ERR_INVALID_ARG : WL_ERR_UNSUPPORTED;
+    if (M < 0 || K < 0) return WL_ERR_INVALID_ARG;
+    if (path != WL_PATH_AUTO && path != WL_PATH_DECODE && path != WL_PATH_GEMM)
+        return WL_ERR_INVALID_ARG;
+    for (int i = 0; i < P; ++i) {
+        const wl_proj &q = projs[i];
+        if (q.N < 0 || q.r < 0) return WL_ERR_INVALID_ARG;
+        if (q.r > WL_MAX_RANK) return WL_ERR_UNSUPPORTED;
+        if (M > 0 && q.N > 0) {
+            if (!q.y || !q.s || (K > 0 && !q.W0)) return WL_ERR_INVALID_ARG;
+            if (q.r > 0 && K > 0 && (!q.U || !q.V)) return WL_ERR_INVALID_ARG;
+        }
+    }
+    if (M > 0 && K > 0 && !x) return WL_ERR_INVALID_ARG;
+    if (K % 8 != 0) return WL_ERR_ALIGNMENT;
+    if (M > 0 && K > 0) {
+        if (!aligned16(x)) return WL_ERR_ALIGNMENT;
+        for (int i = 0; i < P; ++i)
+            if (projs[i].N > 0 && !aligned16(projs[i].W0)) return WL_ERR_ALIGNMENT;
+    }
+    if (path == WL_PATH_DECODE && M > WL_DECODE_MAX_M) return WL_ERR_UNSUPPORTED;
+    return WL_OK;
+}
+
+int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// ------------------------------------------------------------------ paths --
+wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                     cudaStream_t stream) {
+    DecodeParams dp;
+    std::memset(&dp, 0, sizeof dp);
+    int total = 0, tblk = 0, t_off = 0, r_max = 0, nseg = 0;
+    bool u_bulk = true, lowrank = false;
+    for (int i = 0; i < P; ++i) {
+        const wl_proj &q = projs[i];
+        if (q.N == 0) continue;
+        DecodeSeg &sg = dp.seg[nseg++];
+        sg.W0 = reinterpret_cast<const __nv_bfloat16 *>(q.W0);
+        sg.s = q.s;
+        sg.U = reinterpret_cast<const __nv_bfloat16 *>(q.U);
+        sg.V = reinterpret_cast<const __nv_bfloat16 *>(q.V);
+        sg.y = reinterpret_cast<__nv_bfloat16 *>(q.y);
+        sg.N = q.N;
+        sg.r = q.r;
+        sg.t_off = t_off;
+        sg.row_begin = total;
+        sg.tblk_begin = tblk;
+        total += q.N;
+        if (q.r > 0) {
+            lowrank = true;
+            tblk += decode_t_blocks(K);
+            t_off += q.r;
+            r_max = std::max(r_max, q.r);
+            if (q.r % 8 != 0 || !aligned16(q.U)) u_bulk = false;
+        }
+    }
+    if (total == 0) return WL_OK;
+    dp.nseg = nseg;
+    dp.M = M;
+    dp.K = K;
+    dp.total_rows = total;
+    dp.t_ld = t_off;
+    dp.r_max = r_max;
+    dp.u_bulk = u_bulk ? 1 : 0;
+    dp.has_lowrank = lowrank ? 1 : 0;
+    dp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    dp.counters = pool.words + 8;
+    dp.status = pool.words;
+    dp.timeout_ns = kWaitLimitNs;
+    if (lowrank) {
+        void *T = nullptr, *Tp = nullptr;
+        wl_status st = scratch(pool, kSlotT, (size_t)M * t_off * sizeof(float), &T);
+        if (st != WL_OK) return st;
+        st = scratch(pool, kSlotTPart, (size_t)tblk * M * r_max * sizeof(float), &Tp);
+        if (st != WL_OK) return st;
+        dp.T = static_cast<float *>(T);
+        dp.Tpart = static_cast<float *>(Tp);
+    }
+    return from_cuda(launch_decode(dp, pool.num_sms, stream));
+}
+
+wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                   cudaStream_t stream) {
+    // Column layout of T: each projection with r > 0 gets round_up(r, 64) columns.
+    int t_cols = 0;
+    int t_col[kMaxSeg] = {};
+    for (int i = 0; i < P; ++i) {
+        t_col[i] = t_cols;
+        if (projs[i].N > 0 && projs[i].r > 0) t_cols += round_up(projs[i].r, 64);
+    }
+    __nv_bfloat16 *T = nullptr;
+    wl_status st;
+    if (t_cols > 0) {
+        void *vt = nullptr, *t = nullptr;
+        if ((st = scratch(pool, kSlotVt, (size_t)t_cols * K * 2, &vt)) != WL_OK) return st;
+        if ((st = scratch(pool, kSlotT, (size_t)M * t_cols * 2, &t)) != WL_OK) return st;
+        __nv_bfloat16 *Vt = static_cast<__nv_bfloat16 *>(vt);
+        T = static_cast<__nv_bfloat16 *>(t);
+        for (int i = 0; i < P; ++i) {
+            const wl_proj &q = projs[i];
+            if (q.N == 0 || q.r == 0) continue;
+            cudaError_t e = launch_transpose_v(reinterpret_cast<const __nv_bfloat16 *>(q.V), K, q.r,
+                                               round_up(q.r, 64), Vt + (size_t)t_col[i] * K, stream);
+            if (e != cudaSuccess) return WL_ERR_CUDA;
+        }
+        // T = x V for all projections at once (plain GEMM against the stacked V^T).
+        GemmParams tp;
+        std::memset(&tp, 0, sizeof tp);
+        const int bn = t_cols >= 256 ? 256 : t_cols;
+        if ((st = make_map(&tp.tm_a, x, K, M, K, kGemmBM)) != WL_OK) return st;
+        tp.tm_t = tp.tm_a;
+        if ((st = make_map(&tp.tm_b[0], Vt, K, t_cols, K, bn)) != WL_OK) return st;
+        tp.tm_u[0] = tp.tm_b[0];
+        tp.nseg = 1;
+        tp.M = M;
+        tp.K = K;
+        tp.BN = bn;
+        tp.num_m_tiles = (M + kGemmBM - 1) / kGemmBM;
+        tp.seg[0].s = nullptr;
+        tp.seg[0].y = T;
+        tp.seg[0].N = t_cols;
+        tp.seg[0].ldy = t_cols;
+        tp.seg[0].lr_blocks = 0;
+        tp.seg[0].tile_begin = 0;
+        tp.num_tiles = tp.num_m_tiles * ((t_cols + bn - 1) / bn);
+        tp.status = pool.words;
+        tp.timeout_ns = kWaitLimitNs;
+        if (launch_gemm(tp, pool.num_sms, stream) != cudaSuccess) return WL_ERR_CUDA;
+    }
+
+    GemmParams gp;
+    std::memset(&gp, 0, sizeof gp);
+    const int bn = kGemmMaxBN;
+    if ((st = make_map(&gp.tm_a, x, K, M, K, kGemmBM)) != WL_OK) return st;
+    if (t_cols > 0) {
+        if ((st = make_map(&gp.tm_t, T, t_cols, M, t_cols, kGemmBM)) != WL_OK) return st;
+    } else {
+        gp.tm_t = gp.tm_a;
+    }
+    gp.M = M;
+    gp.K = K;
+    gp.BN = bn;
+    gp.num_m_tiles = (M + kGemmBM - 1) / kGemmBM;
+    int tiles = 0, nseg = 0;
+    for (int i = 0; i < P; ++i) {
+        const wl_proj &q = projs[i];
+        if (q.N == 0) continue;
+        const int sidx = nseg++;
+        if ((st = make_map(&gp.tm_b[sidx], q.W0, K, q.N, K, bn)) != WL_OK) return st;
+        GemmSeg &sg = gp.seg[sidx];
+        sg.s = q.s;
+        sg.y = reinterpret_cast<__nv_bfloat16 *>(q.y);
+        sg.N = q.N;
+        sg.ldy = q.N;
+        sg.t_col = t_col[i];
+        sg.tile_begin = tiles;
+        tiles += gp.num_m_tiles * ((q.N + bn - 1) / bn);
+        if (q.r > 0) {
+            const int r_pad = round_up(q.r, 64);
+            sg.lr_blocks = r_pad / 64;
+            if (q.r % 8 == 0 && aligned16(q.U)) {
+                if ((st = make_map(&gp.tm_u[sidx], q.U, q.r, q.N, q.r, bn)) != WL_OK) return st;
+            } else {
+                void *up = nullptr;
+                if ((st = scratch(pool, kSlotUPad0 + sidx, (size_t)q.N * r_pad * 2, &up)) != WL_OK)
+                    return st;
+                if (launch_pad_u(reinterpret_cast<const __nv_bfloat16 *>(q.U), q.N, q.r, r_pad,
+                                 static_cast<__nv_bfloat16 *>(up), stream) != cudaSuccess)
+                    return WL_ERR_CUDA;
+                if ((st = make_map(&gp.tm_u[sidx], up, r_pad, q.N, r_pad, bn)) != WL_OK) return st;
+            }
+        } else {
+            sg.lr_blocks = 0;
+            gp.tm_u[sidx] = gp.tm_b[sidx];
+        }
+    }
+    if (tiles == 0) return WL_OK;
+    gp.nseg = nseg;
+    gp.num_tiles = tiles;
+    gp.status = pool.words;
+    gp.timeout_ns = kWaitLimitNs;
+    return from_cuda(launch_gemm(gp, pool.num_sms, stream));
+}
+
+wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, wl_path path,
+                  void *stream_ptr) {
+    wl_status st = validate(x, M, K, projs, P, path);
+    if (st != WL_OK) return st;
+    bool any = false;
+    for (int i = 0; i < P; ++i) any = any || projs[i].N > 0;
+    if (M == 0 || !any) return WL_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if (K == 0) {  // W0 x = 0 and V^T x = 0: y = 0
+        for (int i = 0; i < P; ++i)
+            if (projs[i].N > 0 &&
+                cudaMemsetAsync(projs[i].y, 0, (size_t)M * projs[i].N * 2, stream) != cudaSuccess)
+                return WL_ERR_CUDA;
+        return WL_OK;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevicePool *pool = nullptr;
+    if ((st = pool_for_current_device(&pool)) != WL_OK) return st;
+    if (path == WL_PATH_AUTO) path = M <= WL_DECODE_MAX_M ? WL_PATH_DECODE : WL_PATH_GEMM;
+    return path == WL_PATH_DECODE ? run_decode(*pool, x, M, K, projs, P, stream)
+                                  : run_gemm(*pool, x, M, K, projs, P, stream);
+}
+
+}  // namespace
+}  // namespace wl
+
+extern "C" {
+
+wl_status wl_linear_forward(const wl_bf16 *x, const wl_bf16 *W0, const float *s, const wl_bf16 *U,
+                            const wl_bf16 *V, wl_bf16 *y, int M, int N, int K, int r, void *stream) {
+    wl_proj p;
+    p.W0 = W0;
+    p.s = s;
+    p.U = U;
+    p.V = V;
+    p.y = y;
+    p.N = N;
+    p.r = r;
+    return wl::forward(x, M, K, &p, 1, WL_PATH_AUTO, stream);
+}
+
+wl_status wl_stacked_forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                             void *stream) {
+    return wl::forward(x, M, K, projs, P, WL_PATH_AUTO, stream);
+}
+
+wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, wl_path path,
+                        void *stream) {
+    return wl::forward(x, M, K, projs, P, path, stream);
+}
+
+const char *wl_status_string(wl_status s) {
+    switch (s) {
+        case WL_OK: return "ok";
+        case WL_ERR_INVALID_ARG: return "invalid argument";
+        case WL_ERR_ALIGNMENT: return "misaligned argument (K % 8 != 0 or pointer not 16-byte aligned)";
+        case WL_ERR_UNSUPPORTED: return "unsupported (rank, projection count, path or device)";
+        case WL_ERR_CUDA: return "CUDA error";
+        case WL_ERR_TIMEOUT: return "device-side wait timed out";
+        case WL_ERR_NOMEM: return "out of device memory";
+    }
+    return "unknown status";
+}
+
+wl_status wl_last_device_status(void *stream) {
+    std::lock_guard<std::mutex> lock(wl::g_mu);
+    wl::DevicePool *pool = nullptr;
+    wl_status st = wl::pool_for_current_device(&pool);
+    if (st != WL_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WL_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, pool->words, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return WL_ERR_CUDA;
+    if (cudaMemset(pool->words, 0, sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
+    return static_cast<wl_status>(word);
+}
+
+wl_status wl_wait_probe(long long limit_ns, void *stream) {
+    if (limit_ns <= 0 || limit_ns > 1000000000LL) return WL_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(wl::g_mu);
+    wl::DevicePool *pool = nullptr;
+    wl_status st = wl::pool_for_current_device(&pool);
+    if (st != WL_OK) return st;
+    return wl::from_cuda(wl::launch_wait_probe(pool->words + 1, pool->words,
+                                               (unsigned long long)limit_ns,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+int wl_version(void) { return (0 << 16) | 1; }
+
+}  // extern "C"

@@ -1,0 +1,186 @@
+// Host-side decomposition of dense layer weights into theta bundles:
+//   band mean W0, least-squares per-row scale s, truncated SVD of the residual.
+// ("Quality", "Why sharing fails: reconstruction error": the band-mean W0,
+// the per-layer residual weight - s.W0 and its rank-r delta; "Add a new model
+// architecture", "Decompose HF weights", step 4.)
+//
+// The SVD is a one-sided Jacobi (Hestenes) iteration in fp64 over the columns
+// of the residual or of its transpose, whichever has fewer columns: pairs of
+// columns are rotated until all pairs are orthogonal; the column norms are then
+// the singular values and the accumulated rotation gives the other side.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <numeric>
+#include <vector>
+
+#include "../../include/wl.h"
+
+namespace {
+
+// A is m x n column-major (n <= m).  On return its columns are mutually
+// orthogonal (A_in Q) and Q (n x n, column-major) holds the rotations.
+void jacobi_orthogonalize(std::vector<double> &A, int m, int n, std::vector<double> &Q) {
+    Q.assign((size_t)n * n, 0.0);
+    for (int i = 0; i < n; ++i) Q[(size_t)i * n + i] = 1.0;
+    const double eps = 1e-15;
+    for (int sweep = 0; sweep < 80; ++sweep) {
+        bool rotated = false;
+        for (int i = 0; i < n - 1; ++i) {
+            double *ai = &A[(size_t)i * m];
+            for (int j = i + 1; j < n; ++j) {
+                double *aj = &A[(size_t)j * m];
+                double alpha = 0, beta = 0, gamma = 0;
+                for (int k = 0; k < m; ++k) {
+                    alpha += ai[k] * ai[k];
+                    beta += aj[k] * aj[k];
+                    gamma += ai[k] * aj[k];
+                }
+                if (gamma == 0.0 || std::fabs(gamma) <= eps * std::sqrt(alpha * beta)) continue;
+                rotated = true;
+                const double zeta = (beta - alpha) / (2.0 * gamma);
+                const double t = (zeta >= 0 ? 1.0 : -1.0) / (std::fabs(zeta) + std::sqrt(1.0 + zeta * zeta));
+                const double c = 1.0 / std::sqrt(1.0 + t * t);
+                const double s = c * t;
+                for (int k = 0; k < m; ++k) {
+                    const double x = ai[k], y = aj[k];
+                    ai[k] = c * x - s * y;
+                    aj[k] = s * x + c * y;
+                }
+                double *qi = &Q[(size_t)i * n], *qj = &Q[(size_t)j * n];
+                for (int k = 0; k < n; ++k) {
+                    const double x = qi[k], y = qj[k];
+                    qi[k] = c * x - s * y;
+                    qj[k] = s * x + c * y;
+                }
+            }
+        }
+        if (!rotated) break;
+    }
+}
+
+// Rank-r truncated SVD of R (N x K, row-major): U = P_r S_r (N x r), V = Q_r (K x r).
+void truncated_svd(const std::vector<double> &R, int N, int K, int r, float *U, float *V) {
+    std::memset(U, 0, sizeof(float) * (size_t)N * r);
+    std::memset(V, 0, sizeof(float) * (size_t)K * r);
+    if (r == 0) return;
+    const bool cols_are_k = K <= N;  // orthogonalise the K columns of R, else the N columns of R^T
+    const int m = cols_are_k ? N : K, n = cols_are_k ? K : N;
+    std::vector<double> A((size_t)m * n);
+    for (int a = 0; a < N; ++a)
+        for (int b = 0; b < K; ++b) {
+            if (cols_are_k)
+                A[(size_t)b * m + a] = R[(size_t)a * K + b];  // column b of R
+            else
+                A[(size_t)a * m + b] = R[(size_t)a * K + b];  // column a of R^T
+        }
+    std::vector<double> Q;
+    jacobi_orthogonalize(A, m, n, Q);
+    std::vector<double> sigma(n);
+    for (int i = 0; i < n; ++i) {
+        double ss = 0;
+        for (int k = 0; k < m; ++k) ss += A[(size_t)i * m + k] * A[(size_t)i * m + k];
+        sigma[i] = std::sqrt(ss);
+    }
+    std::vector<int> order(n);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return sigma[a] > sigma[b]; });
+    const int kk = std::min(r, n);
+    for (int c = 0; c < kk; ++c) {
+        const int i = order[c];
+        const double sg = sigma[i];
+        if (sg == 0.0) continue;  // zero singular value: leave the column zero
+        const double *col = &A[(size_t)i * m];
+        const double *q = &Q[(size_t)i * n];
+        if (cols_are_k) {
+            // R Q = A: column i of A is sigma_i p_i (length N); Q column is v_i (length K)
+            for (int a = 0; a < N; ++a) U[(size_t)a * r + c] = (float)col[a];
+            for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = (float)q[b];
+        } else {
+            // R^T Q = A: R = Q A^T; left vectors are Q columns (length N), right A/sigma (length K)
+            for (int a = 0; a < N; ++a) U[(size_t)a * r + c] = (float)(q[a] * sg);
+            for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = (float)(col[b] / sg);
+        }
+    }
+}
+
+double rel_err_fp64(const float *W, const float *W0, const float *s, const float *U, const float *V,
+                    int N, int K, int r) {
+    double num = 0, den = 0;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            double uv = 0;
+            for (int j = 0; j < r; ++j) uv += (double)U[(size_t)n * r + j] * (double)V[(size_t)k * r + j];
+            const double w = W[(size_t)n * K + k];
+            const double d = w - ((double)s[n] * (double)W0[(size_t)n * K + k] + uv);
+            num += d * d;
+            den += w * w;
+        }
+    return den > 0 ? std::sqrt(num / den) : std::sqrt(num);
+}
+
+}  // namespace
+
+extern "C" {
+
+wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r, const int *band_of_layer,
+                       float *W0, float *s, float *U, float *V, double *rel_err) {
+    if (!W || !W0 || !s || (r > 0 && (!U || !V))) return WL_ERR_INVALID_ARG;
+    if (L < 1 || N < 1 || K < 1 || G < 1 || r < 0) return WL_ERR_INVALID_ARG;
+    try {
+        std::vector<int> band(L);
+        for (int l = 0; l < L; ++l) {
+            band[l] = band_of_layer ? band_of_layer[l] : (int)(((long long)l * G) / L);
+            if (band[l] < 0 || band[l] >= G) return WL_ERR_INVALID_ARG;
+        }
+        const size_t NK = (size_t)N * K;
+        std::vector<double> w0((size_t)G * NK, 0.0);
+        std::vector<int> count(G, 0);
+        for (int l = 0; l < L; ++l) {
+            ++count[band[l]];
+            double *dst = &w0[(size_t)band[l] * NK];
+            const float *src = W + (size_t)l * NK;
+            for (size_t i = 0; i < NK; ++i) dst[i] += src[i];
+        }
+        for (int b = 0; b < G; ++b) {
+            double *dst = &w0[(size_t)b * NK];
+            if (count[b] > 0)
+                for (size_t i = 0; i < NK; ++i) dst[i] /= count[b];
+            for (size_t i = 0; i < NK; ++i) W0[(size_t)b * NK + i] = (float)dst[i];
+        }
+        std::vector<double> R(NK);
+        for (int l = 0; l < L; ++l) {
+            const float *w = W + (size_t)l * NK;
+            const double *b0 = &w0[(size_t)band[l] * NK];
+            float *sl = s + (size_t)l * N;
+            for (int n = 0; n < N; ++n) {
+                double num = 0, den = 0;
+                for (int k = 0; k < K; ++k) {
+                    num += (double)w[(size_t)n * K + k] * b0[(size_t)n * K + k];
+                    den += b0[(size_t)n * K + k] * b0[(size_t)n * K + k];
+                }
+                const double sc = den > 0 ? num / den : 1.0;
+                sl[n] = (float)sc;
+                for (int k = 0; k < K; ++k)
+                    R[(size_t)n * K + k] = (double)w[(size_t)n * K + k] - sc * b0[(size_t)n * K + k];
+            }
+            float *Ul = r > 0 ? U + (size_t)l * N * r : nullptr;
+            float *Vl = r > 0 ? V + (size_t)l * K * r : nullptr;
+            if (r > 0) truncated_svd(R, N, K, r, Ul, Vl);
+            if (rel_err)
+                rel_err[l] = rel_err_fp64(w, W0 + (size_t)band[l] * NK, sl, Ul, Vl, N, K, r);
+        }
+    } catch (const std::bad_alloc &) {
+        return WL_ERR_NOMEM;
+    }
+    return WL_OK;
+}
+
+double wl_relative_frobenius_error(const float *W, const float *W0, const float *s, const float *U,
+                                   const float *V, int N, int K, int r) {
+    if (!W || !W0 || !s || N < 1 || K < 1 || r < 0 || (r > 0 && (!U || !V))) return -1.0;
+    return rel_err_fp64(W, W0, s, U, V, N, K, r);
+}
+
+}  // extern "C"

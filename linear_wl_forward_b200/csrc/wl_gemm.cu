@@ -1,0 +1,319 @@
+// Tensor-core path (any M; chosen for M > 4): a persistent tcgen05 GEMM whose
+// epilogue applies the per-row scale and adds the rank-r term,
+//
+//     y[m][n] = s[n] * sum_k x[m][k] W0[n][k]  +  sum_j T[m][j] U[n][j],
+//     T = x V (computed first by the same kernel in plain mode, bf16 output).
+//
+// Per CTA (one per SM, 192 threads):
+//   warp 0      TMA producer: 128 x 64 tiles of x (or T) and BN x 64 tiles of
+//               W0 (or U), 128-byte swizzled, into a 4-deep ring of 48 KB
+//               stages, completion on mbarriers (no multicast).
+//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
+//               (128 x BN x 16, bf16 in, fp32 accumulate): the K loop over W0
+//               into accumulator A (columns 0..BN-1), then the r/64 low-rank
+//               blocks into accumulator B (columns 256..256+BN-1).  Each stage
+//               is released with tcgen05.commit; the finished tile is signalled
+//               to the epilogue the same way.
+//   warps 2-5   epilogue: tcgen05.ld of both accumulators (one TMEM lane = one
+//               token row per thread), y = s * A + B in fp32, one rounding to
+//               bf16, stores with edge checks.
+// The scale touches only the shared-block product, so the two products keep
+// separate accumulators; U V^T is never formed.
+//
+// Bf16 operands with fp32 accumulation follow "Quality (Gemma 4 31B)", "Kernel
+// optimizations", GEMM path item 2 (bf16 matmuls accumulate in fp32 on the
+// tensor cores); the pages' GEMM path uses two library matmuls per stack, here
+// the low-rank product rides in the same kernel and the same accumulator pass.
+#include "wl_common.cuh"
+#include "wl_internal.h"
+
+namespace wl {
+
+namespace {
+
+constexpr uint32_t kABytes = kGemmBM * kGemmBK * 2;     // 16 KB
+constexpr uint32_t kBBytesMax = kGemmMaxBN * kGemmBK * 2;  // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytesMax;  // 48 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccBCol = 256;
+
+struct TileInfo {
+    int seg, m0, n0;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const GemmParams &p, int t) {
+    int sp = 0;
+    while (sp + 1 < p.nseg && t >= p.seg[sp + 1].tile_begin) ++sp;
+    const int local = t - p.seg[sp].tile_begin;
+    TileInfo ti;
+    ti.seg = sp;
+    ti.m0 = (local % p.num_m_tiles) * kGemmBM;
+    ti.n0 = (local / p.num_m_tiles) * p.BN;
+    return ti;
+}
+
+// All lanes wait; the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const GemmParams &p,
+                                          volatile int *abort_flag) {
+    bool ok = mbar_wait(bar, parity, p.status, p.timeout_ns) && (*abort_flag == 0);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && (threadIdx.x & 31) == 0) *abort_flag = 1;
+    return ok;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    uint8_t *base = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + kGemmStages * kStageBytes);
+    uint64_t *empty = full + kGemmStages;
+    uint64_t *tmem_full = empty + kGemmStages;
+    uint64_t *tmem_empty = tmem_full + 1;
+    uint64_t *drain = tmem_empty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nkb = (p.K + kGemmBK - 1) / kGemmBK;
+    const uint32_t b_bytes = (uint32_t)p.BN * kGemmBK * 2;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGemmStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(tmem_empty, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&p.tm_a);
+        prefetch_tmap(&p.tm_t);
+        for (int i = 0; i < p.nseg; ++i) {
+            prefetch_tmap(&p.tm_b[i]);
+            prefetch_tmap(&p.tm_u[i]);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer ----
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+            const TileInfo ti = tile_info(p, t);
+            const GemmSeg &sg = p.seg[ti.seg];
+            const int total = nkb + sg.lr_blocks;
+            for (int kb = 0; kb < total; ++kb) {
+                const uint32_t slot = it % kGemmStages, ph = (it / kGemmStages) & 1u;
+                if (!warp_wait(&empty[slot], ph ^ 1u, p, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t *sa = base + slot * kStageBytes;
+                    uint8_t *sb = sa + kABytes;
+                    mbar_arrive_expect_tx(&full[slot], kABytes + b_bytes);
+                    if (kb < nkb) {
+                        tma_load_2d(sa, &p.tm_a, kb * kGemmBK, ti.m0, &full[slot]);
+                        tma_load_2d(sb, &p.tm_b[ti.seg], kb * kGemmBK, ti.n0, &full[slot]);
+                    } else {
+                        const int j0 = (kb - nkb) * kGemmBK;
+                        tma_load_2d(sa, &p.tm_t, sg.t_col + j0, ti.m0, &full[slot]);
+                        tma_load_2d(sb, &p.tm_u[ti.seg], j0, ti.n0, &full[slot]);
+                    }
+                }
+                __syncwarp();
+                ++it;
+            }
+        }
+        if (!ok) {
+            // Let the loads already issued land before the CTA exits.
+            const uint32_t inflight = it < (uint32_t)kGemmStages ? it : (uint32_t)kGemmStages;
+            for (uint32_t i = it - inflight; i < it; ++i)
+                mbar_wait(&full[i % kGemmStages], (i / kGemmStages) & 1u, p.status, 1000000ull);
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------- MMA issuer ---
+        const uint32_t idesc = idesc_bf16_f32(kGemmBM, p.BN);
+        uint32_t it = 0, tcount = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+            const TileInfo ti = tile_info(p, t);
+            const GemmSeg &sg = p.seg[ti.seg];
+            const int total = nkb + sg.lr_blocks;
+            if (!warp_wait(tmem_empty, (tcount & 1u) ^ 1u, p, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            for (int kb = 0; kb < total; ++kb) {
+                const uint32_t slot = it % kGemmStages, ph = (it / kGemmStages) & 1u;
+                if (!warp_wait(&full[slot], ph, p, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a_addr = smem_addr(base + slot * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+                    const uint64_t adesc = sw128_kmajor_desc(a_addr);
+                    const uint64_t bdesc = sw128_kmajor_desc(b_addr);
+                    const bool lowrank = kb >= nkb;
+                    const uint32_t d = tmem_base + (lowrank ? kAccBCol : 0u);
+                    const bool first = (kb == 0) || (kb == nkb);
+#pragma unroll
+                    for (int k = 0; k < kGemmBK / 16; ++k) {
+                        // advance 16 elements (32 bytes) along K inside the swizzle row
+                        tc_mma_f16(d, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                   (first && k == 0) ? 0u : 1u);
+                    }
+                    tc_commit(&empty[slot]);
+                }
+                __syncwarp();
+                ++it;
+            }
+            if (!ok) break;
+            if (lane == 0) tc_commit(tmem_full);
+            __syncwarp();
+            ++tcount;
+        }
+        if (!ok) {
+            // Wait for MMAs already issued before TMEM is released.
+            if (lane == 0) tc_commit(drain);
+            __syncwarp();
+            mbar_wait(drain, 0, p.status, 1000000ull);
+        }
+    } else {
+        // ------------------------------------------------------- epilogue ---
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int row_in_tile = q * 32 + lane;
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+        uint32_t tcount = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+            const TileInfo ti = tile_info(p, t);
+            const GemmSeg &sg = p.seg[ti.seg];
+            if (!warp_wait(tmem_full, tcount & 1u, p, abort_flag)) break;
+            tc_fence_after();
+            const int m = ti.m0 + row_in_tile;
+            const bool lr = sg.lr_blocks > 0;
+            const bool vec = ((reinterpret_cast<uintptr_t>(sg.y) & 15u) == 0) && (sg.ldy % 8 == 0);
+            __nv_bfloat16 *yrow = sg.y + (size_t)m * sg.ldy;
+            for (int c = 0; c < p.BN; c += 32) {
+                uint32_t a[32], b[32];
+                tmem_ld32(lane_addr + (uint32_t)c, a);
+                if (lr) tmem_ld32(lane_addr + kAccBCol + (uint32_t)c, b);
+                tmem_ld_wait();
+                const int nb = ti.n0 + c;
+                if (m < p.M && nb < sg.N) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int n = nb + i;
+                        const float sc = (sg.s && n < sg.N) ? __ldg(sg.s + n) : 1.f;
+                        const float acc = __uint_as_float(a[i]);
+                        v[i] = lr ? fmaf(sc, acc, __uint_as_float(b[i])) : sc * acc;
+                    }
+                    if (vec && nb + 32 <= sg.N) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint4 w;
+                            w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+                            w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+                            w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+                            w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+                            dst[i] = w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (nb + i < sg.N) yrow[nb + i] = __float2bfloat16_rn(v[i]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_empty);
+            ++tcount;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+size_t gemm_smem_bytes() { return 1024 + kGemmStages * kStageBytes + 256; }
+
+cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
+    const size_t smem = gemm_smem_bytes();
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    if (grid < 1) return cudaSuccess;
+    gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------- small helpers ---
+__global__ void transpose_v_kernel(const __nv_bfloat16 *__restrict__ V, int K, int r, int r_pad,
+                                   __nv_bfloat16 *__restrict__ Vt) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int k0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+    for (int i = ty; i < 32; i += 8) {
+        const int k = k0 + i, j = j0 + tx;
+        tile[i][tx] = (k < K && j < r) ? V[(size_t)k * r + j] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int j = j0 + i, k = k0 + tx;
+        if (j < r_pad && k < K) Vt[(size_t)j * K + k] = tile[tx][i];
+    }
+}
+
+cudaError_t launch_transpose_v(const __nv_bfloat16 *V, int K, int r, int r_pad, __nv_bfloat16 *Vt,
+                               cudaStream_t stream) {
+    dim3 grid((K + 31) / 32, (r_pad + 31) / 32);
+    transpose_v_kernel<<<grid, dim3(32, 8), 0, stream>>>(V, K, r, r_pad, Vt);
+    return cudaGetLastError();
+}
+
+__global__ void pad_u_kernel(const __nv_bfloat16 *__restrict__ U, int N, int r, int r_pad,
+                             __nv_bfloat16 *__restrict__ Upad) {
+    const size_t total = (size_t)N * r_pad;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const size_t n = i / r_pad;
+        const int j = (int)(i % r_pad);
+        Upad[i] = j < r ? U[n * r + j] : __float2bfloat16_rn(0.f);
+    }
+}
+
+cudaError_t launch_pad_u(const __nv_bfloat16 *U, int N, int r, int r_pad, __nv_bfloat16 *Upad,
+                         cudaStream_t stream) {
+    const size_t total = (size_t)N * r_pad;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 4096) blocks = 4096;
+    if (blocks < 1) return cudaSuccess;
+    pad_u_kernel<<<blocks, 256, 0, stream>>>(U, N, r, r_pad, Upad);
+    return cudaGetLastError();
+}
+
+}  // namespace wl

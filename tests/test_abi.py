@@ -1,0 +1,79 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/wl.h declares, and rejects bad arguments on the host before touching
+CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_wl_forward_b200 as wl
+from linear_wl_forward_b200 import build as wlbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    wlbuild.build()
+    return wl.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "wl.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wl_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(L):
+    names = header_functions()
+    assert "wl_linear_forward" in names and "wl_decompose" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert L.wl_status_string(code)
+    assert L.wl_version() >= 1
+
+
+FAKE = 0x10000  # 16-byte aligned fake device address; never dereferenced
+
+
+def call(L, x=FAKE, W0=FAKE, s=FAKE, U=FAKE, V=FAKE, y=FAKE, M=1, N=8, K=16, r=8):
+    return L.wl_linear_forward(x, W0, s, U, V, y, M, N, K, r, None)
+
+
+def test_host_validation(L):
+    assert call(L, x=None) == 1                  # null x
+    assert call(L, W0=None) == 1
+    assert call(L, s=None) == 1
+    assert call(L, y=None) == 1
+    assert call(L, U=None) == 1                  # r > 0 needs U and V
+    assert call(L, M=-1) == 1
+    assert call(L, N=-2) == 1
+    assert call(L, r=-1) == 1
+    assert call(L, K=12) == 2                    # K % 8 != 0
+    assert call(L, x=FAKE + 2) == 2              # misaligned x
+    assert call(L, W0=FAKE + 8) == 2             # misaligned W0
+    assert call(L, r=wl.MAX_RANK + 1) == 3
+    # empty inputs are a no-op and touch nothing
+    assert call(L, M=0, x=None, y=None) == 0
+    assert call(L, N=0, W0=None, s=None, y=None, U=None, V=None) == 0
+
+
+def test_stacked_validation(L):
+    P = wl.MAX_PROJ + 1
+    arr = (wl._Proj * P)(*[wl._Proj(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 8) for _ in range(P)])
+    assert L.wl_stacked_forward(FAKE, 1, 16, arr, P, None) == 3
+    assert L.wl_stacked_forward(FAKE, 1, 16, arr, 0, None) == 1
+    assert L.wl_stacked_forward(FAKE, 1, 16, None, 1, None) == 1
+    # the decode path serves at most 4 tokens
+    assert L.wl_forward_ex(FAKE, wl.DECODE_MAX_M + 1, 16, arr, 1, wl.PATHS["decode"], None) == 3
+    assert L.wl_forward_ex(FAKE, 1, 16, arr, 1, 7, None) == 1
+
+
+def test_wait_probe_rejects_bad_limit(L):
+    assert L.wl_wait_probe(0, None) == 1
+    assert L.wl_wait_probe(2_000_000_000, None) == 1
