@@ -346,9 +346,17 @@ int decode_t_blocks(int K) { return (K + kTChunk - 1) / kTChunk; }
 template <int M>
 static cudaError_t launch_decode_m(const DecodeParams &p, int num_sms, cudaStream_t stream) {
     const size_t smem = decode_smem_bytes(M);
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    // Opt in to the large shared-memory carve-out once per device.
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        e = cudaFuncSetAttribute(decode_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
 
     if (p.has_lowrank) {
         int tblocks = 0;

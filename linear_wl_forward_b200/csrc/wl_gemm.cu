@@ -262,9 +262,17 @@ size_t gemm_smem_bytes() { return 1024 + kGemmStages * kStageBytes + 256; }
 
 cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
     const size_t smem = gemm_smem_bytes();
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // Opt in to the large shared-memory carve-out once per device.
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
     int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
     if (grid < 1) return cudaSuccess;
     gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(p);
