@@ -115,6 +115,33 @@ wl_status wl_stacked_forward(const wl_bf16 *x, int M, int K, const wl_proj *proj
 wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
                         wl_path path, void *stream);
 
+/* wl_linear_forward for callers that cannot allocate device memory while they
+ * run: code living inside a pre-planned memory arena (an inference engine
+ * whose allocator owns the device), callers under a hard memory budget, or
+ * host threads that must not take the driver's allocation locks on a hot path.
+ * The pages have no counterpart; it exists for these deployments only.
+ *
+ * Same arguments, layouts and conventions as wl_linear_forward, restricted to
+ * the decode path: 1 <= M <= WL_DECODE_MAX_M (M == 0 or N == 0 is a no-op).
+ * Scratch comes from one 4 MiB array in the library's device image that every
+ * GPU loading the library keeps until the process exits; this entry point
+ * never calls cudaMalloc, cudaFree or any allocating routine.  Shapes whose
+ * scratch would exceed it -- 256 B + M*r*4 B + ceil(K/128)*M*r*4 B, each
+ * rounded up to 256 B, above 4 MiB -- return WL_ERR_UNSUPPORTED, as does
+ * M > WL_DECODE_MAX_M.
+ *  - The first call on each device resolves the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array, which keeps the previous call's contents;
+ *    each call clears the parts that must start at zero on its own stream.
+ *    Calls that overlap on the GPU (different streams or host threads) race on
+ *    the array: serialise them.
+ *  - A device-side wait that times out here is recorded in the array's own
+ *    status word, not in the word wl_last_device_status() reads. */
+wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *W0, const float *s,
+                                    const wl_bf16 *U, const wl_bf16 *V, wl_bf16 *y,
+                                    int M, int N, int K, int r, void *stream);
+
 /* Host-side decomposition of L dense layer weights into theta bundles
  * ("Quality", "Why sharing fails": band-mean W0, per-row scale s, low-rank
  * residual; "Add a new model architecture", "Decompose HF weights" step 4).
