@@ -79,11 +79,11 @@ typedef struct {
  * so tests and benchmarks can exercise each kernel on any shape. */
 typedef enum {
     WL_PATH_AUTO = 0,
-    WL_PATH_DECODE = 1, /* streaming CUDA-core kernel, 1 <= M <= WL_DECODE_MAX_M */
+    WL_PATH_DECODE = 1, /* weight-streaming kernel (bulk copies + warp MMA), 1 <= M <= WL_DECODE_MAX_M */
     WL_PATH_GEMM = 2    /* tcgen05 tensor-core GEMM with the fused low-rank epilogue */
 } wl_path;
 
-#define WL_DECODE_MAX_M 4
+#define WL_DECODE_MAX_M 16
 
 /* y = s (.) (W0 x) + U (V^T x) for one projection of one layer
  * ("Add a new model architecture", introduction; the delta is never
@@ -125,10 +125,12 @@ wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, in
  * the decode path: 1 <= M <= WL_DECODE_MAX_M (M == 0 or N == 0 is a no-op).
  * Scratch comes from one 4 MiB array in the library's device image that every
  * GPU loading the library keeps until the process exits; this entry point
- * never calls cudaMalloc, cudaFree or any allocating routine.  Shapes whose
- * scratch would exceed it -- 256 B + M*r*4 B + ceil(K/128)*M*r*4 B, each
- * rounded up to 256 B, above 4 MiB -- return WL_ERR_UNSUPPORTED, as does
- * M > WL_DECODE_MAX_M.
+ * never calls cudaMalloc, cudaFree or any allocating routine.  The scratch a
+ * call needs is 256 B of counters plus, when V is large enough that the CTAs
+ * share the work of V^T x, (grid+1)*M*r*4 B of partial sums (grid <= the SM
+ * count: 149*M*r*4 B on a 148-SM B200).  A call needing more than 4 MiB
+ * returns WL_ERR_UNSUPPORTED, as do M > WL_DECODE_MAX_M and shapes the decode
+ * kernel cannot take (M rounded up to 8, times r, above 12288).
  *  - The first call on each device resolves the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
  *    before any stream capture.

@@ -13,7 +13,66 @@
 #include "wl_internal.h"
 
 namespace wl {
+
 namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up through the runtime so that the
+// library needs no libcuda at link time.
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+}  // namespace
+
+wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
+                        uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return WL_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
+}
+
+wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                        uint32_t b2) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return WL_ERR_CUDA;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    const cuuint32_t box[3] = {b0, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
+}
+
+namespace {
+
+// GEMM operand maps: box_rows x 64 elements.
+wl_status make_map(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
+                   uint32_t box_rows) {
+    return encode_map_2d(m, ptr, cols, rows, ld, 64, box_rows);
+}
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per device-side wait
 constexpr int kMaxDevices = 64;
@@ -76,42 +135,6 @@ wl_status scratch(DevicePool &p, int slot, size_t bytes, void **out) {
     return WL_OK;
 }
 
-// ------------------------------------------------------------ tensor maps --
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
-
-// 2-D bf16 map: `rows` x `cols` elements, row stride `ld` elements, box
-// box_rows x 64 elements (128 B, swizzled 128 B).  Out-of-range reads give 0.
-wl_status make_map(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
-                   uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return WL_ERR_CUDA;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {ld * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
-                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
-}
-
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ------------------------------------------------------------- validation --
@@ -145,12 +168,11 @@ wl_status validate(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 // ------------------------------------------------------------------ paths --
-wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
-                     cudaStream_t stream) {
-    DecodeParams dp;
+// Fills the decode parameters of a call; false if no projection has rows.
+bool build_decode_params(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                         DecodeParams &dp) {
     std::memset(&dp, 0, sizeof dp);
-    int total = 0, tblk = 0, t_off = 0, r_max = 0, nseg = 0;
-    bool u_bulk = true, lowrank = false;
+    int total = 0, t_off = 0, nseg = 0;
     for (int i = 0; i < P; ++i) {
         const wl_proj &q = projs[i];
         if (q.N == 0) continue;
@@ -163,40 +185,36 @@ wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_
         sg.N = q.N;
         sg.r = q.r;
         sg.t_off = t_off;
-        sg.row_begin = total;
-        sg.tblk_begin = tblk;
         total += q.N;
-        if (q.r > 0) {
-            lowrank = true;
-            tblk += decode_t_blocks(K);
-            t_off += q.r;
-            r_max = std::max(r_max, q.r);
-            if (q.r % 8 != 0 || !aligned16(q.U)) u_bulk = false;
-        }
+        t_off += q.r;
     }
-    if (total == 0) return WL_OK;
+    if (total == 0) return false;
     dp.nseg = nseg;
     dp.M = M;
     dp.K = K;
-    dp.total_rows = total;
     dp.t_ld = t_off;
-    dp.r_max = r_max;
-    dp.u_bulk = u_bulk ? 1 : 0;
-    dp.has_lowrank = lowrank ? 1 : 0;
     dp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-    dp.counters = pool.words + 8;
-    dp.status = pool.words;
     dp.timeout_ns = kWaitLimitNs;
-    if (lowrank) {
-        void *T = nullptr, *Tp = nullptr;
-        wl_status st = scratch(pool, kSlotT, (size_t)M * t_off * sizeof(float), &T);
+    return true;
+}
+
+// Returns WL_ERR_UNSUPPORTED if the shape cannot take the decode kernel.
+wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                     cudaStream_t stream) {
+    static thread_local DecodeParams dp;  // large (tensor maps); kept off the stack
+    if (!build_decode_params(x, M, K, projs, P, dp)) return WL_OK;
+    DecodePlan plan;
+    wl_status st0 = plan_decode(dp, pool.num_sms, &plan);
+    if (st0 != WL_OK) return st0;
+    dp.status = pool.words;
+    dp.sync = reinterpret_cast<unsigned int *>(pool.words + 8);
+    if (plan.tpart_bytes) {
+        void *tp = nullptr;
+        wl_status st = scratch(pool, kSlotTPart, plan.tpart_bytes, &tp);
         if (st != WL_OK) return st;
-        st = scratch(pool, kSlotTPart, (size_t)tblk * M * r_max * sizeof(float), &Tp);
-        if (st != WL_OK) return st;
-        dp.T = static_cast<float *>(T);
-        dp.Tpart = static_cast<float *>(Tp);
+        dp.Tpart = static_cast<float *>(tp);
     }
-    return from_cuda(launch_decode(dp, pool.num_sms, stream));
+    return from_cuda(launch_decode(dp, plan, stream));
 }
 
 wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
@@ -320,7 +338,12 @@ wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, w
     std::lock_guard<std::mutex> lock(g_mu);
     DevicePool *pool = nullptr;
     if ((st = pool_for_current_device(&pool)) != WL_OK) return st;
-    if (path == WL_PATH_AUTO) path = M <= WL_DECODE_MAX_M ? WL_PATH_DECODE : WL_PATH_GEMM;
+    if (path == WL_PATH_AUTO && M <= WL_DECODE_MAX_M) {
+        // The decode kernel declines shapes it cannot hold (before launching
+        // anything); those go to the tensor-core GEMM.
+        st = run_decode(*pool, x, M, K, projs, P, stream);
+        return st == WL_ERR_UNSUPPORTED ? run_gemm(*pool, x, M, K, projs, P, stream) : st;
+    }
     return path == WL_PATH_DECODE ? run_decode(*pool, x, M, K, projs, P, stream)
                                   : run_gemm(*pool, x, M, K, projs, P, stream);
 }
@@ -375,7 +398,9 @@ wl_status wl_last_device_status(void *stream) {
     int word = 0;
     if (cudaMemcpy(&word, pool->words, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return WL_ERR_CUDA;
-    if (cudaMemset(pool->words, 0, sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
+    // A kernel that gave up may have left its arrival counters set: clear the
+    // whole word block (status and counters) after an error.
+    if (word != 0 && cudaMemset(pool->words, 0, 64 * sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
     return static_cast<wl_status>(word);
 }
 

@@ -15,12 +15,24 @@ constexpr int kMaxSeg = WL_MAX_PROJ;
 // --------------------------------------------------------------- decode ----
 // Streaming decode kernel: M <= WL_DECODE_MAX_M tokens.  The projections of a
 // stacked call are concatenated into one row space [0, total_rows).
-constexpr int kDecodeKC = 1024;       // K elements per row per stage (2 KB)
-constexpr int kDecodeRowsPerStage = 8;  // one row per consumer warp
-constexpr int kDecodeStages = 8;      // ring depth: 8 x 16 KB in flight per SM
-constexpr int kDecodeRowsCap = 1024;  // rows per CTA (sizes the z partials)
-constexpr int kDecodeThreads = 32 * (kDecodeRowsPerStage + 1);
-constexpr int kTChunk = 128;          // V rows per block of the V^T x kernel
+constexpr int kDecodeWarps = 8;          // consumer warps
+constexpr int kDecodeConsumers = 32 * kDecodeWarps;
+constexpr int kDecodeThreads = kDecodeConsumers;  // every warp feeds its own ring
+constexpr int kDecodeBlockRows = 16;     // rows of one MMA row block
+constexpr int kDecodeChunkK = 64;        // K columns per TMA box (128 B, swizzled)
+constexpr int kDecodeChunkBytes = kDecodeBlockRows * kDecodeChunkK * 2;  // 2 KB
+constexpr int kDecodeSlotChunks = 2;     // chunks per ring slot: 16 rows x 128 columns
+constexpr int kDecodeSlotBytes = kDecodeSlotChunks * kDecodeChunkBytes;  // 4 KB
+constexpr int kDecodeSlotsPerWarp = 4;
+constexpr int kDecodeTMaxFloats = 12288; // M (rounded up to 8) * (sum of ranks) in shared memory
+
+// How a CTA obtains T = V^T x.
+enum DecodeTMode : int {
+    kTNone = 0,   // no projection has a delta
+    kTLocal = 1,  // each CTA forms the T slices its rows need from all of V
+    kTGrid = 2    // each CTA forms partial sums over a K slice; two grid-wide
+                  // arrival counts later every CTA has the T slices it needs
+};
 
 struct DecodeSeg {
     const __nv_bfloat16 *W0;
@@ -31,30 +43,49 @@ struct DecodeSeg {
     int N;
     int r;
     int t_off;      // column offset of this projection's T slice
-    int row_begin;  // first row in the concatenated row space
-    int tblk_begin; // first block of the V^T x kernel for this projection
+    int blk_begin;  // first 16-row block of this projection in the call's block list
 };
 
 struct DecodeParams {
+    CUtensorMap tm_w[kMaxSeg];   // W0: 2-D {K, N}, box {64, 16}, 128-B swizzle
+    CUtensorMap tm_w3[kMaxSeg];  // W0: 3-D {64, N, K/64}, box {64, 16, 4} (when w3d)
+    CUtensorMap tm_u[kMaxSeg];   // U:  2-D {r, N}, box {64, 16} (when u_bulk)
     DecodeSeg seg[kMaxSeg];
     int nseg;
     int M, K;
-    int total_rows;
+    int total_blocks;
     int t_ld;       // row stride of T (sum of ranks)
-    int r_max;
-    int u_bulk;     // all U rows can be moved by 16-byte bulk copies
-    int has_lowrank;
+    int w3d;        // K % 64 == 0: a full slot of W0 is one 3-D box
+    int u_bulk;     // every U is TMA-able (r % 8 == 0, 16-byte aligned)
+    int t_mode;     // DecodeTMode
+    int x_smem;     // x is staged in shared memory (rows padded to x_ld elements)
+    int x_ld;
     const __nv_bfloat16 *x;
-    float *T;       // M x t_ld fp32 (V^T x, written by the V^T x kernel)
-    float *Tpart;   // per-block partial sums, [blocks][M][r_max]
-    int *counters;  // one arrival counter per projection (self-resetting)
+    float *Tpart;   // kTGrid: [grid][M][t_ld] partial sums, then [M][t_ld] final T
+    unsigned int *sync;  // kTGrid: [0], [1] arrival counts, [2] departures; self-resetting
     int *status;
     unsigned long long timeout_ns;
 };
 
-size_t decode_smem_bytes(int M);
-int decode_t_blocks(int K);
-cudaError_t launch_decode(const DecodeParams &p, int num_sms, cudaStream_t stream);
+// Host-side planning shared by every decode entry point.
+struct DecodePlan {
+    int grid;
+    size_t smem;
+    size_t tpart_bytes;  // scratch for kTGrid partial sums and final T (0 otherwise)
+};
+// Fills the block list, the tensor maps, p.w3d, p.u_bulk and p.t_mode; returns
+// WL_ERR_UNSUPPORTED if the shape cannot take the decode path (M above
+// WL_DECODE_MAX_M, or M rounded up to 8 times the sum of ranks above
+// kDecodeTMaxFloats).
+wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan);
+cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
+
+// 2-D / 3-D bf16 tensor maps with 128-byte swizzling; out-of-range reads give 0.
+wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
+                        uint32_t box_cols, uint32_t box_rows);
+wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                        uint32_t b2);
 
 // ----------------------------------------------------------------- GEMM ----
 // tcgen05 GEMM: Y[m][n] = s[n] * sum_k A[m][k] B[n][k] + sum_j T[m][j] U[n][j].

@@ -84,10 +84,6 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
     if (K % 8 != 0) return WL_ERR_ALIGNMENT;
     if (K > 0 && (!aligned16(x) || !aligned16(W0))) return WL_ERR_ALIGNMENT;
     if (M > WL_DECODE_MAX_M) return WL_ERR_UNSUPPORTED;
-    const int tblocks = r > 0 ? decode_t_blocks(K) : 0;
-    const size_t t_bytes = align256((size_t)M * r * sizeof(float));
-    const size_t part_bytes = align256((size_t)tblocks * M * r * sizeof(float));
-    if (kWordsBytes + t_bytes + part_bytes > kScratchBytes) return WL_ERR_UNSUPPORTED;
 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     if (K == 0) return cudaMemsetAsync(y, 0, (size_t)M * N * 2, stream) == cudaSuccess ? WL_OK : WL_ERR_CUDA;
@@ -97,11 +93,7 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
     wl_status st = noalloc_setup(&d);
     if (st != WL_OK) return st;
 
-    // The array keeps the previous call's contents: zero the status word and the
-    // arrival counters, which must start at zero, on the caller's stream.
-    if (cudaMemsetAsync(d->scratch, 0, kWordsBytes, stream) != cudaSuccess) return WL_ERR_CUDA;
-
-    DecodeParams dp;
+    static DecodeParams dp;  // large (tensor maps); guarded by g_noalloc_mu
     std::memset(&dp, 0, sizeof dp);
     DecodeSeg &sg = dp.seg[0];
     sg.W0 = reinterpret_cast<const __nv_bfloat16 *>(W0);
@@ -112,22 +104,23 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
     sg.N = N;
     sg.r = r;
     sg.t_off = 0;
-    sg.row_begin = 0;
-    sg.tblk_begin = 0;
     dp.nseg = 1;
     dp.M = M;
     dp.K = K;
-    dp.total_rows = N;
     dp.t_ld = r;
-    dp.r_max = r;
-    dp.u_bulk = (r > 0 && r % 8 == 0 && aligned16(U)) ? 1 : 0;
-    dp.has_lowrank = r > 0 ? 1 : 0;
     dp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    dp.timeout_ns = 2000000000ull;
+    DecodePlan plan;
+    if ((st = plan_decode(dp, d->num_sms, &plan)) != WL_OK) return st;
+    // Scratch: the word block, then the partial sums of V^T x ((grid+1) x M x r fp32).
+    if (kWordsBytes + align256(plan.tpart_bytes) > kScratchBytes) return WL_ERR_UNSUPPORTED;
+
+    // The array keeps the previous call's contents: zero the status word and the
+    // arrival counters, which must start at zero, on the caller's stream.
+    if (cudaMemsetAsync(d->scratch, 0, kWordsBytes, stream) != cudaSuccess) return WL_ERR_CUDA;
     int *words = reinterpret_cast<int *>(d->scratch);
     dp.status = words;
-    dp.counters = words + 8;
-    dp.T = reinterpret_cast<float *>(d->scratch + kWordsBytes);
-    dp.Tpart = reinterpret_cast<float *>(d->scratch + kWordsBytes + t_bytes);
-    dp.timeout_ns = 2000000000ull;
-    return launch_decode(dp, d->num_sms, stream) == cudaSuccess ? WL_OK : WL_ERR_CUDA;
+    dp.sync = reinterpret_cast<unsigned int *>(words + 8);
+    dp.Tpart = reinterpret_cast<float *>(d->scratch + kWordsBytes);
+    return launch_decode(dp, plan, stream) == cudaSuccess ? WL_OK : WL_ERR_CUDA;
 }

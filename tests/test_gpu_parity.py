@@ -29,7 +29,9 @@ def test_tiny_band_both_layers(path):
 
 # ---------------------------------------------------------- ragged cases ---
 DECODE_CASES = [(1, 1, 8, 0), (1, 37, 24, 5), (2, 300, 1000, 16), (3, 513, 1032, 64),
-                (4, 257, 2056, 256), (1, 2000, 3080, 8), (4, 129, 64, 1024), (2, 64, 8, 3)]
+                (4, 257, 2056, 256), (1, 2000, 3080, 8), (4, 129, 64, 1024), (2, 64, 8, 3),
+                (8, 700, 4104, 24), (13, 333, 520, 256), (16, 2048, 5376, 256), (9, 17, 16, 7),
+                (16, 40, 8, 0), (5, 4000, 136, 1000)]
 GEMM_CASES = [(1, 37, 24, 5), (5, 300, 200, 16), (130, 513, 1000, 64), (257, 255, 136, 72),
               (64, 1024, 520, 256), (200, 77, 64, 0), (129, 600, 2056, 4), (16, 256, 256, 1024),
               (300, 1, 8, 8)]
@@ -45,13 +47,13 @@ def test_gemm_ragged(M, N, K, r):
     check_call(wl_inputs.random_case(23 + M + N + K + r, M, N, K, r), "gemm")
 
 
-@pytest.mark.parametrize("path,M", [("decode", 3), ("gemm", 70)])
+@pytest.mark.parametrize("path,M", [("decode", 3), ("decode", 11), ("gemm", 70)])
 def test_stacked_mixed_ranks(path, M):
     call = wl_inputs.random_case(5, M, [300, 64, 1000], 512, [16, 0, 40], P=3)
     check_call(call, path)
 
 
-@pytest.mark.parametrize("path,M", [("decode", 2), ("gemm", 33)])
+@pytest.mark.parametrize("path,M", [("decode", 2), ("decode", 16), ("gemm", 33)])
 def test_stacked_max_projections(path, M):
     Ns = [40, 8, 130, 256, 17, 300, 64, 9]
     rs = [8, 16, 0, 64, 3, 32, 256, 8]
@@ -60,7 +62,7 @@ def test_stacked_max_projections(path, M):
 
 
 def test_deterministic_repeat():
-    for path, M in (("decode", 4), ("gemm", 150)):
+    for path, M in (("decode", 4), ("decode", 16), ("gemm", 150)):
         call = wl_inputs.random_case(8, M, 700, 1544, 64)
         xd, pd = to_dev(call)
         a = run(call, path, xd, pd)[0]
@@ -129,7 +131,7 @@ def test_bad_arguments_raise():
     with pytest.raises(wl.WLError) as e:
         wl.linear_forward(x, W0, torch.ones(4, device="cuda"), None, None)
     assert e.value.code == 2
-    x = torch.ones(5, 16, dtype=torch.bfloat16, device="cuda")
+    x = torch.ones(wl.DECODE_MAX_M + 1, 16, dtype=torch.bfloat16, device="cuda")
     W0 = torch.ones(4, 16, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(wl.WLError):
         wl.linear_forward(x, W0, torch.ones(4, device="cuda"), None, None, path="decode")

@@ -53,9 +53,8 @@ def test_noalloc_matches_linear_forward_on_two_calls():
     assert MAX_TOL == 2e-2 and FROB_TOL == 5e-3
 
 
-def test_noalloc_rejects_oversized_scratch_and_large_m():
+def test_noalloc_rejects_unsupported_shapes_on_the_host():
     fn = _fn()
-    fake = 0x10000  # 16-byte aligned, never dereferenced: rejected before any launch
-    # rank 1024 at M=4 with K = 32768: partial sums alone exceed the 4 MiB array
-    assert fn(fake, fake, fake, fake, fake, fake, 4, 64, 32768, 1024, None) == 3
+    fake = 0x10000  # 16-byte aligned, never dereferenced: both are rejected before any launch
     assert fn(fake, fake, fake, fake, fake, fake, wl.DECODE_MAX_M + 1, 64, 64, 8, None) == 3
+    assert fn(fake, fake, fake, fake, fake, fake, 1, 64, 64, wl.MAX_RANK + 1, None) == 3
