@@ -176,7 +176,7 @@ bool build_decode_params(const wl_bf16 *x, int M, int K, const wl_proj *projs, i
     for (int i = 0; i < P; ++i) {
         const wl_proj &q = projs[i];
         if (q.N == 0) continue;
-        DecodeSeg &sg = dp.seg[nseg++];
+        DecodeSeg &sg = dp.a.seg[nseg++];
         sg.W0 = reinterpret_cast<const __nv_bfloat16 *>(q.W0);
         sg.s = q.s;
         sg.U = reinterpret_cast<const __nv_bfloat16 *>(q.U);
@@ -189,12 +189,12 @@ bool build_decode_params(const wl_bf16 *x, int M, int K, const wl_proj *projs, i
         t_off += q.r;
     }
     if (total == 0) return false;
-    dp.nseg = nseg;
-    dp.M = M;
-    dp.K = K;
-    dp.t_ld = t_off;
-    dp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-    dp.timeout_ns = kWaitLimitNs;
+    dp.a.nseg = nseg;
+    dp.a.M = M;
+    dp.a.K = K;
+    dp.a.t_ld = t_off;
+    dp.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    dp.a.timeout_ns = kWaitLimitNs;
     return true;
 }
 
@@ -206,13 +206,13 @@ wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_
     DecodePlan plan;
     wl_status st0 = plan_decode(dp, pool.num_sms, &plan);
     if (st0 != WL_OK) return st0;
-    dp.status = pool.words;
-    dp.sync = reinterpret_cast<unsigned int *>(pool.words + 8);
+    dp.a.status = pool.words;
+    dp.a.sync = reinterpret_cast<unsigned int *>(pool.words + 8);
     if (plan.tpart_bytes) {
         void *tp = nullptr;
         wl_status st = scratch(pool, kSlotTPart, plan.tpart_bytes, &tp);
         if (st != WL_OK) return st;
-        dp.Tpart = static_cast<float *>(tp);
+        dp.a.Tpart = static_cast<float *>(tp);
     }
     return from_cuda(launch_decode(dp, plan, stream));
 }

@@ -1,52 +1,59 @@
 // Decode path (M <= 16 tokens): the memory-bound half of the theta-bundle
 // linear, y = s (.) (W0 x) + U (V^T x), as ONE kernel per call.
 //
-// Work split: the output rows of the (stacked) call are cut into blocks of 16
+// Work split.  The output rows of the (stacked) call are cut into blocks of 16
 // rows that never straddle two projections; each CTA (one per SM at most) owns
-// a balanced, contiguous range of blocks.  For every block, each of the eight
-// consumer warps takes a fixed 1/8 share of the 64-column chunks of K (and of
-// the rank r), so all warps stream the same number of bytes.
+// a balanced, contiguous range of blocks (in local T mode, below, the CTAs are
+// first shared out among the projections so that each CTA needs one V).  For
+// every block, each of the eight warps takes a fixed 1/8 share of the
+// 64-column chunks of K (and of the rank r), so all warps stream the same
+// number of bytes.
 //
-// Roles (nine warps):
-//  * producer warp: for each block and each consumer warp, moves the 16 rows x
-//    (up to) 256 columns of W0 -- then of U -- that the warp needs into one of
-//    that warp's two 8 KB shared-memory slots with TMA tensor copies (a single
-//    3-D box {64 columns, 16 rows, 4 chunks} per full slot, 128-byte swizzle,
-//    no multicast), completion counted on mbarriers; 16 slots keep up to 128 KB
-//    in flight per SM.  W0 and U are parameters, so the producer starts at
-//    once, also while the previous kernel in the stream is still running
-//    (programmatic dependent launch).  Rows past the end of a projection are
-//    out of bounds for the copy and arrive as zeros.
-//  * consumer warps: wait for the previous kernel (griddepcontrol.wait: x and
-//    the scratch become valid), form T = V^T x (below), then for each slot run
-//    warp-level tensor-core MMAs (m16n8k16, bf16 in, fp32 accumulate): A = the
-//    16 W0 rows read with ldmatrix through the swizzle (conflict-free), B = x
-//    (token n, column k) loaded from L1/L2.  The U slots go through a second
-//    accumulator with B = T split into bf16 high and low parts, so the
-//    low-rank product keeps fp32-level accuracy.  At the end of a block the
-//    eight warps' accumulators are added in warp order in shared memory and
-//    y = s * (W0 x) + U T is rounded once to bf16.
+// Streaming.  Every warp feeds its own ring of shared-memory slots (a slot is
+// 16 rows x up to 256 columns, one 3-D TMA box {64, 16, chunks} with 128-byte
+// swizzle, or 2-D boxes for a ragged K; no multicast) and refills a slot as
+// soon as it has consumed it, so no warp waits for another to free space.
+// W0 and U are parameters: the whole ring is requested before the kernel waits
+// for the previous kernel in the stream (griddepcontrol.wait), i.e. while that
+// kernel still runs.  Calls whose per-CTA share is small use a compact
+// variant (at most 110 KB of shared memory, two CTAs per SM), so the next
+// call's CTAs become resident beside this call's and stream their W0 during
+// its tail.  Rows past the end of a projection are out of bounds for the copy
+// and arrive as zeros.
+//
+// Arithmetic.  Warp-level tensor-core MMAs (m16n8k16, bf16 in, fp32
+// accumulate): A = 16 W0 rows read with ldmatrix through the swizzle
+// (conflict-free), B = x (token n, column k) from shared memory when it fits,
+// else from L1/L2.  U slots go through a second accumulator with B = T split
+// into bf16 high and low parts, so the low-rank product keeps fp32-level
+// accuracy.  At the end of each step the eight warps' accumulators are added
+// in warp order in shared memory and y = s * (W0 x) + U T is rounded once to
+// bf16.  The stream is HBM-bound (M flop per byte of W0), so these warp MMAs
+// keep the instruction count per byte low without tcgen05's TMEM round trip.
 //
 // T = V^T x is formed inside the same kernel ("cooperative vtx" of the pages'
 // custom op), one of two ways chosen per call on the host:
-//  * local: when every CTA's share of V is small (<= 96 KB), each CTA reads the
-//    V slices its rows need (from L2 after the first touch) and reduces them in
-//    shared memory;
+//  * local: when each CTA's V is small, the CTA reads all of it (bulk-copied
+//    into shared memory before the wait when it fits) and forms its T slices
+//    before the first block: warp MMAs with A = V^T read by ldmatrix.trans,
+//    the warps splitting the k-steps (CUDA cores when V cannot be staged);
 //  * grid: otherwise each CTA forms partial sums over a 1/grid slice of K for
-//    every projection and writes them to scratch; after a grid-wide arrival
-//    count (a bounded wait), CTA c adds up column block c of T over all CTAs
-//    (lanes stride the CTAs, then a fixed shuffle tree); after a second count
-//    every CTA loads the T slices its rows need.  The counters reset
-//    themselves once every CTA is past both counts.
+//    every projection (the warps splitting the 16-column tiles of r) and
+//    writes them to scratch (phase A); one step later it
+//    waits for all CTAs' partials and adds up its 1/grid share of the outputs
+//    over all CTAs (phase B); `lag` steps in it waits for all shares and loads
+//    the slices it needs (phase C).  Meanwhile the W0 stream runs on: in step
+//    t a CTA does the W0 part of its block t and the U part of block t - lag,
+//    keeping z = W0 x of the blocks in between in shared memory.  The counters
+//    reset themselves once every CTA is past both counts.
 // Every sum has a fixed order (no float atomics), so results are reproducible.
 //
 // Prior art: the custom-op kernel on "Quality (Gemma 4 31B)", "Kernel
 // optimizations", custom-op path (128-bit loads, warp-shuffle reductions, one
 // warp per output row, cooperative V^T x, a single block barrier).  Here the
-// W0 stream is staged by TMA, the per-row dot products run on the tensor cores
-// (the stream stays HBM-bound and the instruction count per byte drops by an
-// order of magnitude), rows are spread evenly over all SMs, and consecutive
-// calls overlap through PDL.
+// W0 stream is staged by TMA, the per-row dot products run on the tensor
+// cores, rows are spread evenly over all SMs, and consecutive calls overlap
+// through programmatic dependent launch.
 #include "wl_common.cuh"
 #include "wl_internal.h"
 
@@ -55,31 +62,14 @@ namespace wl {
 namespace {
 
 constexpr int NW = kDecodeWarps;
+constexpr int NTH = kDecodeThreads;
 constexpr int BR = kDecodeBlockRows;
 constexpr int CK = kDecodeChunkK;
-constexpr int SC = kDecodeSlotChunks;
-constexpr int SLOTS = kDecodeSlotsPerWarp;
-constexpr size_t kLocalVBytes = 96 * 1024;
+constexpr size_t kLocalVBytes = 96 * 1024;    // local T when each CTA's V is at most this
 constexpr uint32_t kDecodeMaxSmem = 227 * 1024;
-
-__device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecodeConsumers) : "memory");
-}
-
-// Barrier over the 256 consumer threads that also ORs a predicate across them,
-// so every consumer takes the same abort decision.
-__device__ __forceinline__ bool consumer_any(bool pred) {
-    uint32_t out;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, %2, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(out)
-        : "r"((uint32_t)pred), "n"(kDecodeConsumers)
-        : "memory");
-    return out != 0;
-}
+constexpr uint32_t kSmallSmem = 110 * 1024;   // two CTAs per SM
+constexpr size_t kSmallCtaBytes = 256 * 1024; // W0 + U per CTA up to which a call is small
+constexpr uint32_t kMaxRingBytes = 192 * 1024;
 
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
     unsigned int v;
@@ -91,10 +81,8 @@ __device__ __forceinline__ void red_release_gpu_add(unsigned int *p, unsigned in
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Arrive on a grid-wide counter and wait (bounded) until all CTAs arrived.
-__device__ __forceinline__ bool grid_arrive_wait(unsigned int *ctr, unsigned int expected,
-                                                 const DecodeParams &p) {
-    red_release_gpu_add(ctr, 1u);
+// Wait (bounded) until a grid-wide counter reaches `expected`.
+__device__ __forceinline__ bool grid_wait(const unsigned int *ctr, unsigned int expected, const DecodeArgs &p) {
     const uint64_t t0 = globaltimer_ns();
     uint32_t polls = 0;
     while (ld_acquire_gpu(ctr) < expected) {
@@ -111,7 +99,7 @@ struct Block {
     int sp, row0, nrows;
 };
 
-__device__ __forceinline__ Block block_info(const DecodeParams &p, int b) {
+__device__ __forceinline__ Block block_info(const DecodeArgs &p, int b) {
     int sp = 0;
     while (sp + 1 < p.nseg && b >= p.seg[sp + 1].blk_begin) ++sp;
     Block B;
@@ -121,14 +109,31 @@ __device__ __forceinline__ Block block_info(const DecodeParams &p, int b) {
     return B;
 }
 
-__device__ __forceinline__ int seg_blocks(const DecodeSeg &sg) { return (sg.N + BR - 1) / BR; }
+__host__ __device__ __forceinline__ int seg_blocks(const DecodeSeg &sg) { return (sg.N + BR - 1) / BR; }
 
-__device__ __forceinline__ bool seg_touched(const DecodeSeg &sg, int blk_lo, int blk_hi) {
+// Blocks [lo, hi) of CTA c out of `grid`: an even split of the whole list, or
+// (seg_split) an even split of each projection's blocks over its own CTAs.
+__host__ __device__ inline void cta_blocks(const DecodeArgs &p, int c, int grid, int &lo, int &hi) {
+    if (!p.seg_split) {
+        lo = (int)(((long long)c * p.total_blocks) / grid);
+        hi = (int)(((long long)(c + 1) * p.total_blocks) / grid);
+        return;
+    }
+    int sp = 0;
+    while (sp + 1 < p.nseg && c >= p.seg[sp + 1].cta_begin) ++sp;
+    const DecodeSeg &sg = p.seg[sp];
+    const int nc = (sp + 1 < p.nseg ? p.seg[sp + 1].cta_begin : grid) - sg.cta_begin;
+    const int nb = seg_blocks(sg), j = c - sg.cta_begin;
+    lo = sg.blk_begin + (int)(((long long)j * nb) / nc);
+    hi = sg.blk_begin + (int)(((long long)(j + 1) * nb) / nc);
+}
+
+__host__ __device__ __forceinline__ bool seg_touched(const DecodeSeg &sg, int blk_lo, int blk_hi) {
     return sg.r > 0 && sg.blk_begin < blk_hi && sg.blk_begin + seg_blocks(sg) > blk_lo;
 }
 
 // All lanes wait on the barrier phase; the warp agrees on the outcome.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const DecodeParams &p,
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const DecodeArgs &p,
                                           volatile int *abort_flag) {
     bool ok = mbar_wait(bar, parity, p.status, p.timeout_ns) && (*abort_flag == 0);
     ok = __all_sync(0xffffffffu, ok);
@@ -136,12 +141,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const 
     return ok;
 }
 
-__device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tmap, int c0, int c1, int c2,
-                                            uint64_t *bar) {
+// L2 policy for the streamed operands (W0, U): each byte is read once per
+// call, so those lines go first when L2 needs room and the small, reused data
+// (x, V, s, T scratch, the kernel's own code and parameters) stays cached.
+__device__ __forceinline__ uint64_t stream_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void tma_stream_2d(void *dst_smem, const void *tmap, int c0, int c1, uint64_t *bar,
+                                              uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst_smem)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(pol)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_stream_3d(void *dst_smem, const void *tmap, int c0, int c1, int c2,
+                                              uint64_t *bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar)), "l"(pol)
         : "memory");
 }
 
@@ -170,66 +193,96 @@ __device__ __forceinline__ uint32_t ldg_u32(const __nv_bfloat16 *p) {
     return __ldg(reinterpret_cast<const unsigned int *>(p));
 }
 
-// Chunks [lo, hi) of consumer warp w among n chunks.
-__device__ __forceinline__ void warp_chunks(int n, int w, int &lo, int &hi) {
+// Chunks [lo, hi) of warp w among n chunks.
+__host__ __device__ __forceinline__ void warp_chunks(int n, int w, int &lo, int &hi) {
     lo = (w * n) / NW;
     hi = ((w + 1) * n) / NW;
 }
 
 // Chunks of the rank r that warp w streams: handed out in reverse warp order,
 // so they land first on the warps whose W0 share is one chunk short.
-__device__ __forceinline__ void warp_u_chunks(int r, int w, int &lo, int &hi) {
+__host__ __device__ __forceinline__ void warp_u_chunks(int r, int w, int &lo, int &hi) {
     warp_chunks((r + CK - 1) / CK, NW - 1 - w, lo, hi);
 }
 
-// A warp's position in its sequence of ring copies: slot s of block b, with
-// the block's layout for this warp (W0 chunks are fixed for the call, U chunks
-// depend on the block's projection).
+// A warp's position in its sequence of ring copies.  The CTA's work is a list
+// of steps t = 0 .. nblk + lag - 1; step t holds the W0 part of the CTA's
+// block t (t < nblk) and then the U part of its block t - lag (t >= lag, when
+// that block's projection has a delta).  Every warp walks the same list.
 struct WarpSeq {
-    int b, s;
-    int ns, nw0;       // slots in this block, of which W0 slots
-    int u_lo, u_hi;    // U chunk range in this block
-    int sp, row0, nrows;
+    int t, part, s;  // step, part (0 = W0, 1 = U), slot within the part
+    int ns;          // slots of this part for this warp
+    int sp, row0;    // projection and first row of the part's block
+    int u_lo, u_hi;  // U chunk range (part 1)
 };
 
-__device__ __forceinline__ void seq_load(const DecodeParams &p, int w, int w0_slots, WarpSeq &q) {
-    const Block B = block_info(p, q.b);
+__device__ __forceinline__ void seq_load(const DecodeArgs &p, int w, int w0_slots, int blk_lo, int nblk,
+                                         WarpSeq &q) {
+    q.ns = 0;
+    int b;
+    if (q.part == 0) {
+        if (q.t >= nblk) return;
+        b = blk_lo + q.t;
+    } else {
+        if (q.t < p.lag || q.t - p.lag >= nblk) return;
+        b = blk_lo + q.t - p.lag;
+    }
+    const Block B = block_info(p, b);
     q.sp = B.sp;
     q.row0 = B.row0;
-    q.nrows = B.nrows;
-    q.nw0 = w0_slots;
-    q.u_lo = q.u_hi = 0;
+    if (q.part == 0) {
+        q.ns = w0_slots;
+        return;
+    }
     const int r = p.seg[B.sp].r;
-    if (p.u_bulk && r > 0) warp_u_chunks(r, w, q.u_lo, q.u_hi);
-    q.ns = w0_slots + (q.u_hi - q.u_lo + SC - 1) / SC;
+    if (!p.u_bulk || r == 0) return;
+    warp_u_chunks(r, w, q.u_lo, q.u_hi);
+    q.ns = (q.u_hi - q.u_lo + p.slot_chunks - 1) / p.slot_chunks;
 }
 
-// Moves q to the next slot this warp streams, crossing blocks as needed;
-// false once the CTA's blocks are exhausted.
-__device__ __forceinline__ bool seq_next(const DecodeParams &p, int w, int w0_slots, int blk_hi,
+// Moves q to the next slot this warp streams; false once the list is done.
+__device__ __forceinline__ bool seq_next(const DecodeArgs &p, int w, int w0_slots, int blk_lo, int nblk,
                                          WarpSeq &q) {
+    const int nsteps = nblk + p.lag;
     ++q.s;
     while (q.s >= q.ns) {
-        if (++q.b >= blk_hi) return false;
+        if (q.part == 0) {
+            q.part = 1;
+        } else {
+            q.part = 0;
+            ++q.t;
+        }
+        if (q.t >= nsteps) return false;
         q.s = 0;
-        seq_load(p, w, w0_slots, q);
+        seq_load(p, w, w0_slots, blk_lo, nblk, q);
     }
     return true;
 }
 
+// Positions q at the first slot of the list; false if it is empty.
+__device__ __forceinline__ bool seq_first(const DecodeArgs &p, int w, int w0_slots, int blk_lo, int nblk,
+                                          WarpSeq &q) {
+    q.t = 0;
+    q.part = 0;
+    seq_load(p, w, w0_slots, blk_lo, nblk, q);
+    q.s = -1;
+    return seq_next(p, w, w0_slots, blk_lo, nblk, q);
+}
+
 // One lane: expect the bytes and start the TMA copies of the slot at q.
-__device__ __forceinline__ void issue_slot(const DecodeParams &p, const WarpSeq &q, int w0_lo, int w0_hi,
-                                           uint8_t *dst, uint64_t *bar) {
-    const bool is_u = q.s >= q.nw0;
-    const int c_lo = is_u ? q.u_lo + (q.s - q.nw0) * SC : w0_lo + q.s * SC;
-    const int c_hi = min(is_u ? q.u_hi : w0_hi, c_lo + SC);
+__device__ __forceinline__ void issue_slot(const DecodeParams &P, const DecodeArgs &p, const WarpSeq &q, int w0_lo,
+                                           int w0_hi, uint8_t *dst, uint64_t *bar, uint64_t pol) {
+    const int sc = p.slot_chunks;
+    const bool is_u = q.part == 1;
+    const int c_lo = (is_u ? q.u_lo : w0_lo) + q.s * sc;
+    const int c_hi = min(is_u ? q.u_hi : w0_hi, c_lo + sc);
     mbar_arrive_expect_tx(bar, (uint32_t)(c_hi - c_lo) * kDecodeChunkBytes);
-    if (!is_u && p.w3d && c_hi - c_lo == SC) {
-        tma_load_3d(dst, &p.tm_w3[q.sp], 0, q.row0, c_lo, bar);
+    if (!is_u && p.w3d && c_hi - c_lo == sc) {
+        tma_stream_3d(dst, &P.tm_w3[q.sp], 0, q.row0, c_lo, bar, pol);
     } else {
-        const CUtensorMap *tm = is_u ? &p.tm_u[q.sp] : &p.tm_w[q.sp];
+        const CUtensorMap *tm = is_u ? &P.tm_u[q.sp] : &P.tm_w[q.sp];
         for (int cc = c_lo; cc < c_hi; ++cc)
-            tma_load_2d(dst + (cc - c_lo) * kDecodeChunkBytes, tm, cc * CK, q.row0, bar);
+            tma_stream_2d(dst + (cc - c_lo) * kDecodeChunkBytes, tm, cc * CK, q.row0, bar, pol);
     }
 }
 
@@ -313,201 +366,399 @@ __device__ __forceinline__ void u_chunk(float (&acu)[NT][4], uint32_t cbase, con
     }
 }
 
-// out[m * out_ld + j] = sum_{k0 <= k < k1} V[k][j] x[m][k] for j < r and m < M,
-// computed by the 256 consumer threads (all must call it) on CUDA cores.  x is
-// read from xsrc with row stride xld (shared or global memory).  `red` is
-// shared scratch of 256 * 8 floats; each output is a fixed-order sum.
-template <int MT>
-__device__ void vtx_block(const __nv_bfloat16 *__restrict__ V, int r, int k0, int k1,
-                          const __nv_bfloat16 *xsrc, int xld, int M, float *red, float *out,
-                          int out_ld) {
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int g8 = r >> 3;
-    if (MT <= 8 && (r & 7) == 0 && g8 > 0 && (kDecodeConsumers % g8) == 0) {
-        // 16-byte vectors of 8 columns; thread t always sees column group t % g8
-        // and every (256 / g8)-th row of the slice.
-        const int reps = kDecodeConsumers / g8;
-        const int grp = tid % g8, rep = tid / g8;
-        float acc[MT][8];
+// out[m * out_ld + j] = sum_{k0 <= k < k1} V[k][j] x[m][k] for j < r, m < M,
+// on the tensor cores (m16n8k16, A = V^T read with ldmatrix.trans from the
+// staged rows, B = x, fp32 accumulate): warp w takes the 16-row k-steps
+// w, w + 8, ...; the eight warps' partial sums are added in warp order.  Row
+// k of V is at vs + (k - k0) * r (16-byte aligned rows, r % 8 == 0); rows
+// past k1 may hold anything and are masked.  x is read from xsrc with row
+// stride xld (shared memory when XS).  `red` is shared scratch of
+// NW * 4 * NT * 128 floats.  All threads must call it; ends with a barrier.
+// B fragments of x for the k-step at kb: columns kb + 2q (+1) and kb + 8 + 2q
+// (+1) of token rows nt * 8 + g, zero past k1 (k1 is even, so no pair
+// straddles it) and for rows past M.
+template <int NT, bool XS>
+__device__ __forceinline__ void x_frags(uint32_t (&b)[NT][2], const __nv_bfloat16 *xsrc, int xld, int M, int kb,
+                                        int k1, int g, int q) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[m][e] = 0.f;
-#pragma unroll 8
-        for (int k = k0 + rep; k < k1; k += reps) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(V + (size_t)k * r + grp * 8));
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m < M) {
-                    const float xv = __bfloat162float(xsrc[(size_t)m * xld + k]);
-                    acc[m][0] = fmaf(bf16lo(v.x), xv, acc[m][0]);
-                    acc[m][1] = fmaf(bf16hi(v.x), xv, acc[m][1]);
-                    acc[m][2] = fmaf(bf16lo(v.y), xv, acc[m][2]);
-                    acc[m][3] = fmaf(bf16hi(v.y), xv, acc[m][3]);
-                    acc[m][4] = fmaf(bf16lo(v.z), xv, acc[m][4]);
-                    acc[m][5] = fmaf(bf16hi(v.z), xv, acc[m][5]);
-                    acc[m][6] = fmaf(bf16lo(v.w), xv, acc[m][6]);
-                    acc[m][7] = fmaf(bf16hi(v.w), xv, acc[m][7]);
-                }
-            }
+    for (int nt = 0; nt < NT; ++nt) {
+        const int n = nt * 8 + g;
+        b[nt][0] = b[nt][1] = 0u;
+        if (n < M) {
+            const __nv_bfloat16 *xr = xsrc + (size_t)n * xld + kb + 2 * q;
+            if (kb + 2 * q < k1) b[nt][0] = XS ? *reinterpret_cast<const uint32_t *>(xr) : ldg_u32(xr);
+            if (kb + 8 + 2 * q < k1) b[nt][1] = XS ? *reinterpret_cast<const uint32_t *>(xr + 8) : ldg_u32(xr + 8);
         }
-        // Per token: lanes of a warp sharing a column group (lane % g8) add with
-        // a fixed xor tree, then the remaining copies add in order via `red`.
-        const bool shuffle = g8 < 32;
-        const int nsrc = shuffle ? NW : reps;
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if (m >= M) break;
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = acc[m][e];
-            if (shuffle) {
-                for (int o = 16; o >= g8; o >>= 1)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] += __shfl_xor_sync(0xffffffffu, v[e], o);
-                if (lane < g8)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) red[(w * g8 + lane) * 8 + e] = v[e];
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) red[tid * 8 + e] = v[e];
-            }
-            consumer_sync();
-            for (int j = tid; j < r; j += kDecodeConsumers) {
-                const int gg = j >> 3, e = j & 7;
-                float s = 0.f;
-                for (int q = 0; q < nsrc; ++q) s += red[(gg + q * g8) * 8 + e];
-                out[(size_t)m * out_ld + j] = s;
-            }
-            consumer_sync();
-        }
-    } else if ((r & 1) == 0 && r / 2 <= kDecodeConsumers) {
-        // Column pairs (4-byte loads); (256 / pairs) threads split the rows.
-        const int P2 = r / 2;
-        const int reps = kDecodeConsumers / P2;
-        const int pair = tid % P2, rep = tid / P2;
-        float acc[MT][2];
-#pragma unroll
-        for (int m = 0; m < MT; ++m) acc[m][0] = acc[m][1] = 0.f;
-        if (rep < reps) {
-#pragma unroll 4
-            for (int k = k0 + rep; k < k1; k += reps) {
-                const uint32_t v = ldg_u32(V + (size_t)k * r + 2 * pair);
-                const float v0 = bf16lo(v), v1 = bf16hi(v);
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (m < M) {
-                        const float xv = __bfloat162float(xsrc[(size_t)m * xld + k]);
-                        acc[m][0] = fmaf(v0, xv, acc[m][0]);
-                        acc[m][1] = fmaf(v1, xv, acc[m][1]);
-                    }
-                }
-            }
-        }
-        const bool shuffle = (32 % P2) == 0;  // lanes sharing a pair sit in one warp
-        const int nsrc = shuffle ? NW : reps;
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if (m >= M) break;
-            float v0 = acc[m][0], v1 = acc[m][1];
-            if (shuffle) {
-                for (int o = 16; o >= P2; o >>= 1) {
-                    v0 += __shfl_xor_sync(0xffffffffu, v0, o);
-                    v1 += __shfl_xor_sync(0xffffffffu, v1, o);
-                }
-                if (lane < P2) {
-                    red[(w * P2 + lane) * 2 + 0] = v0;
-                    red[(w * P2 + lane) * 2 + 1] = v1;
-                }
-            } else if (rep < reps) {
-                red[tid * 2 + 0] = v0;
-                red[tid * 2 + 1] = v1;
-            }
-            consumer_sync();
-            for (int j = tid; j < r; j += kDecodeConsumers) {
-                const int pj = j >> 1, e = j & 1;
-                float s = 0.f;
-                for (int q = 0; q < nsrc; ++q) s += red[(pj + q * P2) * 2 + e];
-                out[(size_t)m * out_ld + j] = s;
-            }
-            consumer_sync();
-        }
-    } else {
-        // Odd or very wide ranks: one column per thread per pass.
-        for (int jb = 0; jb < r; jb += kDecodeConsumers) {
-            const int j = jb + tid;
-            if (j < r) {
-                float acc[MT];
-#pragma unroll
-                for (int m = 0; m < MT; ++m) acc[m] = 0.f;
-                for (int k = k0; k < k1; ++k) {
-                    const float v = __bfloat162float(V[(size_t)k * r + j]);
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        if (m < M) acc[m] = fmaf(v, __bfloat162float(xsrc[(size_t)m * xld + k]), acc[m]);
-                }
-                for (int m = 0; m < M; ++m) out[(size_t)m * out_ld + j] = acc[m];
-            }
-        }
-        consumer_sync();
     }
 }
 
+// A fragment of V^T (16 columns j0.. of r x 16 rows kb.. of the staged V)
+// through ldmatrix.trans; elements of rows past k1 are cleared.
+__device__ __forceinline__ void vt_frag(uint32_t (&a)[4], uint32_t v_lane, int r, int k0, int kb, int k1, int j0,
+                                        int q) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(v_lane + (uint32_t)((kb - k0) * r + j0) * 2u));
+    if (kb + 16 > k1) {
+        if (kb + 2 * q >= k1) a[0] = a[1] = 0u;
+        if (kb + 8 + 2 * q >= k1) a[2] = a[3] = 0u;
+    }
+}
+
+template <int NT, bool XS>
+__device__ void vtx_mma(const __nv_bfloat16 *vs, int r, int k0, int k1, const __nv_bfloat16 *xsrc, int xld,
+                        int M, float *red, float *out, int out_ld) {
+    constexpr int JT = 4;  // 16-column tiles of r per pass
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int g = lane >> 2, q = lane & 3;
+    const int nks = (k1 - k0 + 15) >> 4;
+    const int njt = (r + 15) >> 4;
+    // ldmatrix.trans source row (k) and column (j) offsets of this lane
+    const int lk = (lane & 7) + ((lane >> 4) << 3), lj = ((lane >> 3) & 1) << 3;
+    const uint32_t v_lane = smem_addr(vs) + (uint32_t)(lk * r + lj) * 2u;
+    if (njt >= NW || nks < NW) {
+        // Few k-steps or many column tiles (grid-mode slices): warp w takes
+        // the tiles w, w + 8, ... over all k-steps and writes complete sums.
+        for (int jt = w; jt < njt; jt += NW) {
+            const int j0 = jt * 16;
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+            for (int ks = 0; ks < nks; ++ks) {
+                const int kb = k0 + ks * 16;
+                uint32_t b[NT][2], a[4];
+                x_frags<NT, XS>(b, xsrc, xld, M, kb, k1, g, q);
+                vt_frag(a, v_lane, r, k0, kb, k1, j0, q);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], a, b[nt][0], b[nt][1]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int n = nt * 8 + 2 * q, j = j0 + g;
+                if (n < M) {
+                    if (j < r) out[(size_t)n * out_ld + j] = acc[nt][0];
+                    if (j + 8 < r) out[(size_t)n * out_ld + j + 8] = acc[nt][2];
+                }
+                if (n + 1 < M) {
+                    if (j < r) out[(size_t)(n + 1) * out_ld + j] = acc[nt][1];
+                    if (j + 8 < r) out[(size_t)(n + 1) * out_ld + j + 8] = acc[nt][3];
+                }
+            }
+        }
+        __syncthreads();
+        return;
+    }
+    // Many k-steps, few tiles (local mode): warp w takes the k-steps w, w + 8,
+    // ...; the eight warps' partial sums are added in warp order.
+    for (int jt0 = 0; jt0 < r; jt0 += 16 * JT) {
+        float acc[JT][NT][4];
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[jt][nt][e] = 0.f;
+        for (int ks = w; ks < nks; ks += NW) {
+            const int kb = k0 + ks * 16;
+            uint32_t b[NT][2];
+            x_frags<NT, XS>(b, xsrc, xld, M, kb, k1, g, q);
+#pragma unroll
+            for (int jt = 0; jt < JT; ++jt) {
+                const int j0 = jt0 + jt * 16;
+                if (j0 >= r) break;
+                uint32_t a[4];
+                vt_frag(a, v_lane, r, k0, kb, k1, j0, q);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[jt][nt], a, b[nt][0], b[nt][1]);
+            }
+        }
+        // partial sums of this pass: red[((w * JT + jt) * NT + nt) * 128 + lane * 4 + e]
+#pragma unroll
+        for (int jt = 0; jt < JT; ++jt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                *reinterpret_cast<float4 *>(red + ((size_t)(w * JT + jt) * NT + nt) * 128 + lane * 4) =
+                    make_float4(acc[jt][nt][0], acc[jt][nt][1], acc[jt][nt][2], acc[jt][nt][3]);
+        __syncthreads();
+        const int ncol = min(16 * JT, r - jt0);
+        for (int i = threadIdx.x; i < M * ncol; i += NTH) {
+            const int m = i / ncol, jj = i - m * ncol;
+            const int jt = jj >> 4, jr = jj & 15;
+            const int nt = m >> 3, col = m & 7;
+            const int fl = (jr & 7) * 4 + (col >> 1), fe = (jr >> 3) * 2 + (col & 1);
+            float s = 0.f;
+            for (int ww = 0; ww < NW; ++ww) s += red[((size_t)(ww * JT + jt) * NT + nt) * 128 + fl * 4 + fe];
+            out[(size_t)m * out_ld + jt0 + jj] = s;
+        }
+        __syncthreads();
+    }
+}
+
+// The same sum on CUDA cores, for V rows that are not staged (unaligned, odd
+// rank, or no room): V row k at V + (k - vk0) * r (global or shared), element
+// loads.  Token by token; the threads sharing a column split the rows and add
+// their partial sums in thread order through `red` (NTH floats).  All threads
+// must call it; ends with a barrier.
+__device__ __noinline__ void vtx_cores(const __nv_bfloat16 *V, int vk0, int r, int k0, int k1,
+                                       const __nv_bfloat16 *xsrc, int xld, int M, float *red, float *out,
+                                       int out_ld) {
+    const int tid = threadIdx.x;
+    const int cols = r < NTH ? r : NTH;
+    const int parts = NTH / cols;
+    const int jl = tid % cols, part = tid / cols;
+    for (int m = 0; m < M; ++m) {
+        for (int jb = 0; jb < r; jb += cols) {
+            const int j = jb + jl;
+            float s = 0.f;
+            if (part < parts && j < r)
+                for (int k = k0 + part; k < k1; k += parts)
+                    s = fmaf(__bfloat162float(V[(size_t)(k - vk0) * r + j]),
+                             __bfloat162float(xsrc[(size_t)m * xld + k]), s);
+            red[tid] = s;
+            __syncthreads();
+            if (tid < cols && jb + tid < r) {
+                float t = 0.f;
+                for (int pp = 0; pp < parts; ++pp) t += red[pp * cols + tid];
+                out[(size_t)m * out_ld + jb + tid] = t;
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// V rows [k0, k1) of projection sp that CTA c reads to form T (empty if none):
+// all of K for the projections its rows touch (local mode), or its 1/grid
+// share of the 16-row k-steps of K for every projection with a delta (grid
+// mode).
+__host__ __device__ inline void v_range(const DecodeArgs &p, int sp, int c, int grid, int blk_lo, int blk_hi,
+                                        int &k0, int &k1) {
+    const DecodeSeg &sg = p.seg[sp];
+    k0 = k1 = 0;
+    if (sg.r == 0) return;
+    if (p.t_mode == kTLocal) {
+        if (seg_touched(sg, blk_lo, blk_hi)) k1 = p.K;
+    } else if (p.t_mode == kTGrid) {
+        // whole 16-row k-steps, so slice edges never split a column pair
+        const int nks = (p.K + 15) / 16;
+        k0 = 16 * (int)(((long long)c * nks) / grid);
+        k1 = 16 * (int)(((long long)(c + 1) * nks) / grid);
+        k0 = k0 < p.K ? k0 : p.K;
+        k1 = k1 < p.K ? k1 : p.K;
+    }
+}
+
+// Local mode: T slices of the projections this CTA's rows touch into Ts.
+template <int NT, bool XS>
+__device__ void form_t_local(const DecodeArgs &p, int blk_lo, int blk_hi, const __nv_bfloat16 *xsrc, int xld,
+                             const uint8_t *vs, float *red, float *Ts) {
+    uint32_t off = 0;
+    for (int sp = 0; sp < p.nseg; ++sp) {
+        const DecodeSeg &sg = p.seg[sp];
+        if (!seg_touched(sg, blk_lo, blk_hi)) continue;
+        if (p.v_stage)
+            vtx_mma<NT, XS>(reinterpret_cast<const __nv_bfloat16 *>(vs + off), sg.r, 0, p.K, xsrc, xld, p.M, red,
+                            Ts + sg.t_off, p.t_ld);
+        else
+            vtx_cores(sg.V, 0, sg.r, 0, p.K, xsrc, xld, p.M, red, Ts + sg.t_off, p.t_ld);
+        off += (uint32_t)p.K * (uint32_t)sg.r * 2u;
+    }
+}
+
+// Grid mode, phase A: partial sums over this CTA's K slice for every
+// projection with a delta (zeros for an empty slice: all partials are added),
+// then arrive on the first counter.
+template <int NT, bool XS>
+__device__ void grid_t_partials(const DecodeArgs &p, int blk_lo, int blk_hi, const __nv_bfloat16 *xsrc,
+                                int xld, const uint8_t *vs, float *red) {
+    const int n_out = p.M * p.t_ld;
+    uint32_t off = 0;
+    for (int sp = 0; sp < p.nseg; ++sp) {
+        const DecodeSeg &sg = p.seg[sp];
+        if (sg.r == 0) continue;
+        int k0, k1;
+        v_range(p, sp, blockIdx.x, gridDim.x, blk_lo, blk_hi, k0, k1);
+        float *out = p.Tpart + (size_t)blockIdx.x * n_out + sg.t_off;
+        if (p.v_stage)
+            vtx_mma<NT, XS>(reinterpret_cast<const __nv_bfloat16 *>(vs + off), sg.r, k0, k1, xsrc, xld, p.M, red,
+                            out, p.t_ld);
+        else
+            vtx_cores(sg.V, 0, sg.r, k0, k1, xsrc, xld, p.M, red, out, p.t_ld);
+        off += (uint32_t)(k1 - k0) * (uint32_t)sg.r * 2u;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) red_release_gpu_add(&p.sync[0], 1u);
+}
+
+// Grid mode, phase B: once every CTA's partials are in, add up this CTA's
+// 1/grid share of the outputs over all CTAs (lanes stride the CTAs, then a
+// fixed xor tree; four outputs per warp at a time) into the final T, then
+// arrive on the second counter.  Returns the CTA's common verdict.
+__device__ bool grid_t_reduce(const DecodeArgs &p, volatile int *abort_flag) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const unsigned grid = gridDim.x;
+    bool fail = tid == 0 && !grid_wait(&p.sync[0], grid, p);
+    if (__syncthreads_or(fail || *abort_flag != 0)) return false;
+    const int n_out = p.M * p.t_ld;
+    float *Tfin = p.Tpart + (size_t)grid * n_out;
+    const int o_lo = (int)(((long long)blockIdx.x * n_out) / grid);
+    const int o_hi = (int)(((long long)(blockIdx.x + 1) * n_out) / grid);
+    for (int o0 = o_lo + 4 * w; o0 < o_hi; o0 += 4 * NW) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        for (unsigned c = lane; c < grid; c += 32) {
+            const float *src = p.Tpart + (size_t)c * n_out + o0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (o0 + i < o_hi) s[i] += __ldcg(src + i);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[i] = warp_sum(s[i]);
+        if (lane == 0)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (o0 + i < o_hi) Tfin[o0 + i] = s[i];
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) red_release_gpu_add(&p.sync[1], 1u);
+    return true;
+}
+
+// Grid mode, phase C: once every share is in, load the T slices this CTA's
+// rows need into Ts.  The last CTA past both counts resets the counters for
+// the next call (nobody polls them any more).
+__device__ bool grid_t_load(const DecodeArgs &p, int blk_lo, int blk_hi, float *Ts, volatile int *abort_flag) {
+    const int tid = threadIdx.x;
+    const unsigned grid = gridDim.x;
+    bool fail = tid == 0 && !grid_wait(&p.sync[1], grid, p);
+    if (__syncthreads_or(fail || *abort_flag != 0)) return false;
+    const float *Tfin = p.Tpart + (size_t)grid * p.M * p.t_ld;
+    for (int sp = 0; sp < p.nseg; ++sp) {
+        const DecodeSeg &sg = p.seg[sp];
+        if (!seg_touched(sg, blk_lo, blk_hi)) continue;
+        for (int i = tid; i < p.M * sg.r; i += NTH) {
+            const int m = i / sg.r, j = i - m * sg.r;
+            const size_t o = (size_t)m * p.t_ld + sg.t_off + j;
+            Ts[o] = __ldcg(Tfin + o);
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && atomicAdd(&p.sync[2], 1u) == grid - 1) {
+        atomicExch(&p.sync[0], 0u);
+        atomicExch(&p.sync[1], 0u);
+        atomicExch(&p.sync[2], 0u);
+    }
+    return true;
+}
+
+constexpr uint32_t kArgsBytes = (uint32_t)((sizeof(DecodeArgs) + 15) & ~size_t(15));
+
 struct SmemLayout {
-    uint32_t ring_bytes, ts_off, red_off, xs_off, bar_off, flag_off, total;
+    uint32_t slot_bytes, ring_bytes, ts_off, red_off, xs_off, vs_off, zs_off, bar_off, flag_off, total;
 };
 
-// The ring starts at a 1024-byte boundary (the 128-byte swizzle repeats every
-// 1024 bytes); total includes the slack for that alignment.
-__host__ __device__ inline SmemLayout smem_layout(int NT, int t_ld, uint32_t x_bytes) {
-    const int MT = 8 * NT;
+// Shared memory opens with the copy of the arguments; the ring starts at the
+// next 1024-byte boundary (the 128-byte swizzle repeats every 1024 bytes) and
+// the offsets below are relative to it; total includes the slack for that
+// alignment.
+__host__ __device__ inline SmemLayout smem_layout(const DecodeArgs &p, int NT) {
     SmemLayout L;
-    L.ring_bytes = (uint32_t)NW * SLOTS * kDecodeSlotBytes;
+    L.slot_bytes = (uint32_t)p.slot_chunks * kDecodeChunkBytes;
+    L.ring_bytes = (uint32_t)NW * p.slots * L.slot_bytes;
     L.ts_off = L.ring_bytes;
-    L.red_off = L.ts_off + (((uint32_t)(MT * t_ld) * 4u + 127u) & ~127u);
-    const uint32_t vtx_red = (uint32_t)kDecodeConsumers * 8u * 4u;
-    const uint32_t epi_red = 2u * NW * 32u * 8u * (uint32_t)NT * 4u;
-    L.xs_off = L.red_off + (vtx_red > epi_red ? vtx_red : epi_red);
-    L.bar_off = L.xs_off + ((x_bytes + 127u) & ~127u);
-    L.flag_off = L.bar_off + 2u * NW * SLOTS * 8u;
-    L.total = L.flag_off + 16u + 1024u;
+    L.red_off = L.ts_off + (((uint32_t)(p.M * p.t_ld) * 4u + 127u) & ~127u);
+    const uint32_t epi_red = 2u * NW * 32u * 8u * (uint32_t)NT * 4u;  // two step buffers
+    const uint32_t vtx_red = (uint32_t)NW * 4u * (uint32_t)NT * 128u * 4u;
+    L.xs_off = L.red_off + (epi_red > vtx_red ? epi_red : vtx_red);
+    const uint32_t x_bytes = p.x_smem ? (uint32_t)p.M * p.x_ld * 2u : 0u;
+    L.vs_off = L.xs_off + ((x_bytes + 127u) & ~127u);
+    const uint32_t v_bytes = p.v_stage ? (uint32_t)p.v_bytes : 0u;
+    L.zs_off = L.vs_off + ((v_bytes + 127u) & ~127u);
+    const uint32_t z_bytes = p.lag > 0 ? (uint32_t)(p.lag + 1) * BR * p.M * 4u : 0u;
+    L.bar_off = L.zs_off + ((z_bytes + 127u) & ~127u);
+    L.flag_off = L.bar_off + (uint32_t)(NW * p.slots + 1) * 8u;
+    L.total = L.flag_off + 16u + 1024u + kArgsBytes;  // + the copy of the arguments, before the ring
     return L;
+}
+
+// What step t of a CTA holds (see WarpSeq).
+struct Step {
+    bool has_w, has_u;  // W0 part of block t / U part of block t - lag exist
+    Block bw, bu;
+    int rw, ru;         // ranks of those blocks' projections
+};
+
+__device__ __forceinline__ Step step_info(const DecodeArgs &p, int blk_lo, int nblk, int t) {
+    Step S;
+    S.has_w = t < nblk;
+    S.has_u = t >= p.lag && t - p.lag < nblk;
+    S.bw = S.has_w ? block_info(p, blk_lo + t) : Block{0, 0, 0};
+    S.bu = S.has_u ? block_info(p, blk_lo + t - p.lag) : Block{0, 0, 0};
+    S.rw = S.has_w ? p.seg[S.bw.sp].r : 0;
+    S.ru = S.has_u ? p.seg[S.bu.sp].r : 0;
+    return S;
+}
+
+// The scales this thread applies in step t: for y of block t (written in
+// this step when it has no delta or lag is 0) and of block t - lag.
+__device__ __forceinline__ void step_scales(const DecodeArgs &p, const Step &S, int tid, float &sc_w,
+                                            float &sc_u) {
+    const int M = p.M;
+    sc_w = sc_u = 0.f;
+    if (S.has_w && (S.rw == 0 || p.lag == 0) && tid < S.bw.nrows * M)
+        sc_w = __ldg(p.seg[S.bw.sp].s + S.bw.row0 + tid / M);
+    if (S.has_u && S.ru > 0 && p.lag > 0 && tid < S.bu.nrows * M)
+        sc_u = __ldg(p.seg[S.bu.sp].s + S.bu.row0 + tid / M);
 }
 
 }  // namespace
 
-template <int NT, bool XS>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
-    decode_kernel(const __grid_constant__ DecodeParams p) {
-    constexpr int MT = 8 * NT;
+template <int NT, bool XS, bool SMALL>
+__global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid_constant__ DecodeParams P) {
     // The next kernel in the stream may launch now; it waits for this grid
     // before it reads anything this grid writes.
     pdl_launch_dependents();
 
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_addr = smem_addr(smem_raw);
-    uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-    const SmemLayout L = smem_layout(NT, p.t_ld, XS ? (uint32_t)(p.M * p.x_ld * 2) : 0u);
+    // All threads copy the arguments into shared memory (one round of
+    // parallel loads); everything below reads that copy.
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(&P.a);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(smem_raw);
+        for (int i = threadIdx.x; i < (int)(sizeof(DecodeArgs) / 4); i += NTH) dst[i] = src[i];
+    }
+    __syncthreads();
+    const DecodeArgs &p = *reinterpret_cast<const DecodeArgs *>(smem_raw);
+    const uint32_t raw_addr = smem_addr(smem_raw) + kArgsBytes;
+    uint8_t *smem = smem_raw + kArgsBytes + ((1024u - (raw_addr & 1023u)) & 1023u);
+    const SmemLayout L = smem_layout(p, NT);
     uint8_t *ring = smem;
     float *Ts = reinterpret_cast<float *>(smem + L.ts_off);    // [M][t_ld]
-    float *red = reinterpret_cast<float *>(smem + L.red_off);
+    float *red = reinterpret_cast<float *>(smem + L.red_off);  // step sums; T scratch before the steps
     __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(smem + L.xs_off);  // [M][x_ld]
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);  // [NW][SLOTS]
+    uint8_t *vs = smem + L.vs_off;                             // staged V rows
+    float *zs = reinterpret_cast<float *>(smem + L.zs_off);    // [lag + 1][16 * M]: z awaiting U T
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);  // [NW][slots]
+    const int SLOTS = p.slots;
+    uint64_t *vbar = full + NW * SLOTS;  // V rows staged
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.flag_off);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-    const int blk_lo = (int)(((long long)blockIdx.x * p.total_blocks) / gridDim.x);
-    const int blk_hi = (int)(((long long)(blockIdx.x + 1) * p.total_blocks) / gridDim.x);
-    const int K = p.K, M = p.M;
+    int blk_lo, blk_hi;
+    cta_blocks(p, blockIdx.x, gridDim.x, blk_lo, blk_hi);
+    const int nblk = blk_hi - blk_lo, nsteps = nblk + p.lag;
+    const int K = p.K, M = p.M, SC = p.slot_chunks;
 
     if (tid == 0) {
-        for (int i = 0; i < NW * SLOTS; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < NW * SLOTS + 1; ++i) mbar_init(&full[i], 1);
         *abort_flag = 0;
         fence_barrier_init();
         for (int i = 0; i < p.nseg; ++i) {
-            prefetch_tmap(&p.tm_w[i]);
-            if (p.w3d) prefetch_tmap(&p.tm_w3[i]);
-            if (p.u_bulk && p.seg[i].r > 0) prefetch_tmap(&p.tm_u[i]);
+            prefetch_tmap(&P.tm_w[i]);
+            if (p.w3d) prefetch_tmap(&P.tm_w3[i]);
+            if (p.u_bulk && p.seg[i].r > 0) prefetch_tmap(&P.tm_u[i]);
         }
     }
     __syncthreads();
@@ -517,114 +768,69 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     warp_chunks((K + CK - 1) / CK, warp, w0_lo, w0_hi);
     const int w0_slots = (w0_hi - w0_lo + SC - 1) / SC;
 
-    // Each warp feeds its own SLOTS-deep ring: W0 and U are parameters, so the
-    // first copies go out before waiting for the previous kernel.
+    // Each warp feeds its own ring; W0, U, V and s are parameters, so the V
+    // rows for T and the whole ring are requested before waiting for the
+    // previous kernel.
     uint64_t *my_full = full + warp * SLOTS;
-    uint8_t *my_ring = ring + (size_t)warp * SLOTS * kDecodeSlotBytes;
+    uint8_t *my_ring = ring + (size_t)warp * SLOTS * L.slot_bytes;
+    const uint64_t pol = stream_policy();
     WarpSeq iq;  // issue position
-    iq.b = blk_lo;
-    iq.s = -1;
-    bool more = blk_lo < blk_hi;
-    if (more) {
-        seq_load(p, warp, w0_slots, iq);
-        iq.s = 0;
-        while (iq.s >= iq.ns) {  // blocks where this warp has nothing to stream
-            if (++iq.b >= blk_hi) {
-                more = false;
-                break;
-            }
-            seq_load(p, warp, w0_slots, iq);
+    bool more = seq_first(p, warp, w0_slots, blk_lo, nblk, iq);
+    uint32_t issued = 0;
+    int isl = 0;  // ring slot of the next copy
+    auto issue_next = [&]() {
+        if (lane == 0)
+            issue_slot(P, p, iq, w0_lo, w0_hi, my_ring + (size_t)isl * L.slot_bytes, &my_full[isl], pol);
+        ++issued;
+        if (++isl == SLOTS) isl = 0;
+        more = seq_next(p, warp, w0_slots, blk_lo, nblk, iq);
+    };
+    if (p.v_stage && tid == 0) {
+        uint32_t total = 0;
+        for (int sp = 0; sp < p.nseg; ++sp) {
+            int k0, k1;
+            v_range(p, sp, blockIdx.x, gridDim.x, blk_lo, blk_hi, k0, k1);
+            total += (uint32_t)(k1 - k0) * (uint32_t)p.seg[sp].r * 2u;
+        }
+        mbar_arrive_expect_tx(vbar, total);
+        uint32_t off = 0;
+        for (int sp = 0; sp < p.nseg; ++sp) {
+            int k0, k1;
+            v_range(p, sp, blockIdx.x, gridDim.x, blk_lo, blk_hi, k0, k1);
+            const uint32_t bytes = (uint32_t)(k1 - k0) * (uint32_t)p.seg[sp].r * 2u;
+            if (bytes) bulk_load(vs + off, p.seg[sp].V + (size_t)k0 * p.seg[sp].r, bytes, vbar);
+            off += bytes;
         }
     }
-    uint32_t issued = 0;
-    for (int i = 0; i < SLOTS && more; ++i) {
-        if (lane == 0) issue_slot(p, iq, w0_lo, w0_hi, my_ring + (size_t)i * kDecodeSlotBytes, &my_full[i]);
-        ++issued;
-        more = seq_next(p, warp, w0_slots, blk_hi, iq);
-    }
+    while (more && issued < (uint32_t)SLOTS) issue_next();
+    Step S = step_info(p, blk_lo, nblk, 0);
+    float sc_w, sc_u;
+    step_scales(p, S, tid, sc_w, sc_u);
 
     pdl_wait_primary();  // the previous kernel is done: x and the scratch are ours
-    bool ok = true;
     const __nv_bfloat16 *xsrc = p.x;
     int xld = K;
     if (XS) {
         // x (M x K) into shared memory, rows padded so B-fragment reads are
-        // conflict-free; read once from L2 instead of once per row block.
+        // conflict-free; read once from L2 instead of once per block.
         const int vpr = K / 8;  // 16-byte vectors per row
-        for (int i = tid; i < M * vpr; i += kDecodeConsumers) {
+        for (int i = tid; i < M * vpr; i += NTH) {
             const int m = i / vpr, v = i - m * vpr;
             *reinterpret_cast<uint4 *>(xs + (size_t)m * p.x_ld + v * 8) =
                 __ldg(reinterpret_cast<const uint4 *>(p.x + (size_t)m * K + v * 8));
         }
-        consumer_sync();
+        __syncthreads();
         xsrc = xs;
         xld = p.x_ld;
     }
 
-    // ---- T = V^T x for the projections this CTA's rows belong to ----
-    if (p.t_mode == kTLocal) {
-        for (int sp = 0; sp < p.nseg; ++sp) {
-            const DecodeSeg &sg = p.seg[sp];
-            if (seg_touched(sg, blk_lo, blk_hi))
-                vtx_block<MT>(sg.V, sg.r, 0, K, xsrc, xld, M, red, Ts + sg.t_off, p.t_ld);
-        }
-    } else if (p.t_mode == kTGrid) {
-        // (1) all partials written -> (2) CTA c adds column block c over all
-        // CTAs into Tfin -> (3) every CTA loads the T slices it needs.
-        const unsigned grid = gridDim.x;
-        const int n_out = M * p.t_ld;
-        float *Tfin = p.Tpart + (size_t)grid * n_out;
-        const int k_lo = (int)(((long long)blockIdx.x * K) / grid);
-        const int k_hi = (int)(((long long)(blockIdx.x + 1) * K) / grid);
-        float *part = p.Tpart + (size_t)blockIdx.x * n_out;
-        for (int sp = 0; sp < p.nseg; ++sp) {
-            const DecodeSeg &sg = p.seg[sp];
-            if (sg.r > 0)
-                vtx_block<MT>(sg.V, sg.r, k_lo, k_hi, xsrc, xld, M, red, part + sg.t_off, p.t_ld);
-        }
-        __threadfence();
-        consumer_sync();
-        bool fail = tid == 0 && !grid_arrive_wait(&p.sync[0], grid, p);
-        ok = !consumer_any(fail || *abort_flag != 0);
-        if (ok) {
-            const int o_lo = (int)(((long long)blockIdx.x * n_out) / grid);
-            const int o_hi = (int)(((long long)(blockIdx.x + 1) * n_out) / grid);
-            for (int o = o_lo + warp; o < o_hi; o += NW) {
-                float s = 0.f;
-                for (unsigned c = lane; c < grid; c += 32) s += __ldcg(p.Tpart + (size_t)c * n_out + o);
-                s = warp_sum(s);
-                if (lane == 0) Tfin[o] = s;
-            }
-            __threadfence();
-            consumer_sync();
-            fail = tid == 0 && !grid_arrive_wait(&p.sync[1], grid, p);
-            ok = !consumer_any(fail || *abort_flag != 0);
-        }
-        if (ok) {
-            for (int sp = 0; sp < p.nseg; ++sp) {
-                const DecodeSeg &sg = p.seg[sp];
-                if (!seg_touched(sg, blk_lo, blk_hi)) continue;
-                for (int i = tid; i < M * sg.r; i += kDecodeConsumers) {
-                    const int m = i / sg.r, j = i - m * sg.r;
-                    const size_t o = (size_t)m * p.t_ld + sg.t_off + j;
-                    Ts[o] = __ldcg(Tfin + o);
-                }
-            }
-            consumer_sync();
-            if (tid == 0) {
-                // The last CTA past both arrival counts resets the counters
-                // for the next call (nobody polls them any more).
-                if (atomicAdd(&p.sync[2], 1u) == grid - 1) {
-                    atomicExch(&p.sync[0], 0u);
-                    atomicExch(&p.sync[1], 0u);
-                    atomicExch(&p.sync[2], 0u);
-                }
-            }
-        }
-    }
-    ok = !consumer_any(!ok || *abort_flag != 0);
+    bool ok = true;
+    if (p.t_mode != kTNone && p.v_stage)
+        ok = !__syncthreads_or(!mbar_wait(vbar, 0, p.status, p.timeout_ns) || *abort_flag != 0);
+    if (ok && p.t_mode == kTLocal) form_t_local<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red, Ts);
+    if (ok && p.t_mode == kTGrid) grid_t_partials<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red);
+    const int t_reduce = p.lag >= 2 ? 1 : 0;  // grid mode: step of phase B (phase C is at step lag)
 
-    // ---- row blocks: z = W0 x and U T on the tensor cores ----
     const int g = lane >> 2, q = lane & 3;          // fragment row / column-pair index
     const int lrow = lane & 15, lhalf = lane >> 4;  // ldmatrix source row / k half
     const uint32_t ring_s = smem_addr(my_ring) + (uint32_t)lrow * 128u;
@@ -643,79 +849,94 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         xs_lane[nt] = smem_addr(xs) + (uint32_t)((nn * p.x_ld + 2 * q) * 2);
         xg_lane[nt] = p.x + (size_t)nn * K + 2 * q;
     }
+
     uint32_t consumed = 0;
+    int csl = 0;       // ring slot of the next copy to consume
+    uint32_t cph = 0;  // its barrier phase parity
+    // Consumed the slot: every lane's fragments were used by the MMAs above;
+    // order those generic-proxy reads before the async-proxy refill.
+    auto release_slot = [&]() {
+        ++consumed;
+        if (++csl == SLOTS) {
+            csl = 0;
+            cph ^= 1u;
+        }
+        __syncwarp();
+        if (more) {
+            if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue_next();
+        }
+    };
+
     int buf = 0;
-    for (int b = blk_lo; b < blk_hi && ok; ++b) {
-        WarpSeq cq;
-        cq.b = b;
-        cq.s = 0;
-        seq_load(p, warp, w0_slots, cq);
-        const DecodeSeg &sg = p.seg[cq.sp];
-        // The scale of the output this thread writes at the end of the block,
-        // fetched now so its latency hides behind the block's MMAs.
-        const int n_out = cq.nrows * M;
-        const float sc = tid < n_out ? __ldg(sg.s + cq.row0 + tid / M) : 0.f;
+    for (int t = 0; t < nsteps && ok; ++t) {
+        if (p.t_mode == kTGrid) {
+            if (t == t_reduce) ok = grid_t_reduce(p, abort_flag);
+            if (ok && t == p.lag) ok = grid_t_load(p, blk_lo, blk_hi, Ts, abort_flag);
+            if (!ok) break;
+        }
         float acc[NT][4], acu[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[nt][e] = acu[nt][e] = 0.f;
 
-        for (int s = 0; s < cq.ns; ++s) {
-            const uint32_t sidx = consumed % SLOTS, ph = (consumed / SLOTS) & 1u;
-            if (!warp_wait(&my_full[sidx], ph, p, abort_flag)) {
-                ok = false;  // the warps decide together at the block barrier
+        // ---- W0 part of block t: z = W0 x ----
+        for (int s = 0; S.has_w && s < w0_slots && ok; ++s) {
+            if (!warp_wait(&my_full[csl], cph, p, abort_flag)) {
+                ok = false;  // the warps decide together at the step barrier
                 break;
             }
-            const uint32_t sbase = ring_s + sidx * (uint32_t)kDecodeSlotBytes;
-            if (s < cq.nw0) {
-                const int c_lo = w0_lo + s * SC;
-                const int nch = min(SC, w0_hi - c_lo);
-                for (int cc = 0; cc < nch; ++cc) {
-                    const uint32_t cbase = sbase + (uint32_t)cc * kDecodeChunkBytes;
-                    const int kk0 = (c_lo + cc) * CK;
-                    if (kk0 + CK <= K)
-                        w0_chunk<NT, XS, true>(acc, cbase, swz, kk0, K, nvalid, xs_lane, xg_lane);
-                    else
-                        w0_chunk<NT, XS, false>(acc, cbase, swz, kk0, K, nvalid, xs_lane, xg_lane);
-                }
-            } else {
-                const int c_lo = cq.u_lo + (s - cq.nw0) * SC;
-                const int nch = min(SC, cq.u_hi - c_lo);
-                for (int cc = 0; cc < nch; ++cc)
-                    u_chunk<NT>(acu, sbase + (uint32_t)cc * kDecodeChunkBytes, swz, (c_lo + cc) * CK, sg.r,
-                                Ts + sg.t_off, p.t_ld, g, q, nvalid);
+            const uint32_t sbase = ring_s + (uint32_t)csl * L.slot_bytes;
+            const int c_lo = w0_lo + s * SC;
+            const int nch = min(SC, w0_hi - c_lo);
+            for (int cc = 0; cc < nch; ++cc) {
+                const uint32_t cbase = sbase + (uint32_t)cc * kDecodeChunkBytes;
+                const int kk0 = (c_lo + cc) * CK;
+                if (kk0 + CK <= K)
+                    w0_chunk<NT, XS, true>(acc, cbase, swz, kk0, K, nvalid, xs_lane, xg_lane);
+                else
+                    w0_chunk<NT, XS, false>(acc, cbase, swz, kk0, K, nvalid, xs_lane, xg_lane);
             }
-            ++consumed;
-            // Refill this slot with the warp's next copy: every lane's fragments
-            // were consumed by the MMAs above; order those generic-proxy reads
-            // before the async-proxy write.
-            __syncwarp();
-            if (more) {
-                if (lane == 0) {
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    issue_slot(p, iq, w0_lo, w0_hi, my_ring + (size_t)sidx * kDecodeSlotBytes, &my_full[sidx]);
-                }
-                ++issued;
-                more = seq_next(p, warp, w0_slots, blk_hi, iq);
-            }
+            release_slot();
         }
 
-        // delta without TMA (odd rank or unaligned U): A fragments from global
-        if (ok && !p.u_bulk && sg.r > 0) {
+        // ---- U part of block t - lag: U T ----
+        const bool u_part = S.has_u && S.ru > 0;
+        const DecodeSeg &sgu = p.seg[S.bu.sp];
+        if (u_part && p.u_bulk && ok) {
+            int u_lo, u_hi;
+            warp_u_chunks(S.ru, warp, u_lo, u_hi);
+            const int nu = (u_hi - u_lo + SC - 1) / SC;
+            for (int s = 0; s < nu; ++s) {
+                if (!warp_wait(&my_full[csl], cph, p, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sbase = ring_s + (uint32_t)csl * L.slot_bytes;
+                const int c_lo = u_lo + s * SC;
+                const int nch = min(SC, u_hi - c_lo);
+                for (int cc = 0; cc < nch; ++cc)
+                    u_chunk<NT>(acu, sbase + (uint32_t)cc * kDecodeChunkBytes, swz, (c_lo + cc) * CK, S.ru,
+                                Ts + sgu.t_off, p.t_ld, g, q, nvalid);
+                release_slot();
+            }
+        }
+        if (u_part && !p.u_bulk && ok) {
+            // delta without TMA (odd rank or unaligned U): A fragments from global
             int lo, hi;
-            warp_u_chunks(sg.r, warp, lo, hi);
+            warp_u_chunks(S.ru, warp, lo, hi);
             lo *= CK;
-            hi = min(sg.r, hi * CK);
-            const float *T = Ts + sg.t_off;
+            hi = min(S.ru, hi * CK);
+            const float *T = Ts + sgu.t_off;
             for (int j0 = lo; j0 < hi; j0 += 16) {
                 uint32_t a[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int row = g + 8 * (h & 1), j = j0 + 2 * q + 8 * (h >> 1);
                     float u0 = 0.f, u1 = 0.f;
-                    if (row < cq.nrows) {
-                        const __nv_bfloat16 *ur = sg.U + (size_t)(cq.row0 + row) * sg.r;
+                    if (row < S.bu.nrows) {
+                        const __nv_bfloat16 *ur = sgu.U + (size_t)(S.bu.row0 + row) * S.ru;
                         if (j < hi) u0 = __bfloat162float(ur[j]);
                         if (j + 1 < hi) u1 = __bfloat162float(ur[j + 1]);
                     }
@@ -737,7 +958,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             }
         }
 
-        // ---- add the eight warps' accumulators; y = s * z + U T ----
+        // ---- add the eight warps' accumulators ----
         float *rb = red + (size_t)buf * NW * 32 * 8 * NT;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -745,11 +966,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             dst[0] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
             dst[1] = make_float4(acu[nt][0], acu[nt][1], acu[nt][2], acu[nt][3]);
         }
-        if (consumer_any(!ok || *abort_flag != 0)) {
+        if (__syncthreads_or(!ok || *abort_flag != 0)) {
             ok = false;  // every warp leaves together
             break;
         }
-        if (tid < n_out) {  // n_out <= 16 * 16 = the thread count
+        const Step cur = S;
+        const float cur_sc_w = sc_w, cur_sc_u = sc_u;
+        if (t + 1 < nsteps) {
+            // the next step's blocks and scales, loaded now so their latency
+            // hides behind this step's epilogue and the next step's MMAs
+            S = step_info(p, blk_lo, nblk, t + 1);
+            step_scales(p, S, tid, sc_w, sc_u);
+        }
+        if (tid < BR * M) {  // 16 * M <= the thread count
             const int row = tid / M, n = tid - row * M;
             const int nt = n >> 3, tc = n & 7;
             const int fl = (row & 7) * 4 + (tc >> 1);  // fragment lane
@@ -761,97 +990,228 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 z += f[fe];
                 d += f[4 + fe];
             }
-            sg.y[(size_t)n * sg.N + cq.row0 + row] = __float2bfloat16_rn(fmaf(sc, z, d));
+            if (cur.has_w && row < cur.bw.nrows) {
+                const DecodeSeg &sg = p.seg[cur.bw.sp];
+                if (cur.rw > 0 && p.lag > 0)
+                    zs[(t % (p.lag + 1)) * BR * M + tid] = z;  // y once U T of the block is in
+                else
+                    sg.y[(size_t)n * sg.N + cur.bw.row0 + row] =
+                        __float2bfloat16_rn(fmaf(cur_sc_w, z, p.lag == 0 ? d : 0.f));
+            }
+            if (cur.has_u && cur.ru > 0 && p.lag > 0 && row < cur.bu.nrows) {
+                const DecodeSeg &sg = p.seg[cur.bu.sp];
+                const float zu = zs[((t - p.lag) % (p.lag + 1)) * BR * M + tid];
+                sg.y[(size_t)n * sg.N + cur.bu.row0 + row] = __float2bfloat16_rn(fmaf(cur_sc_u, zu, d));
+            }
         }
         buf ^= 1;
     }
 
     // Copies still in flight (only after an abort) land before the CTA exits.
-    for (uint32_t i = consumed; i < issued; ++i)
-        mbar_wait(&my_full[i % SLOTS], (i / SLOTS) & 1u, p.status, 1000000ull);
-    __syncthreads();
+    while (consumed < issued) {
+        mbar_wait(&my_full[csl], cph, p.status, 1000000ull);
+        ++consumed;
+        if (++csl == SLOTS) {
+            csl = 0;
+            cph ^= 1u;
+        }
+    }
+    if (tid == 0 && p.v_stage) mbar_wait(vbar, 0, p.status, 1000000ull);
 }
 
 // ------------------------------------------------------------------ host ---
-wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
-    if (p.M < 1 || p.M > WL_DECODE_MAX_M || p.K < 8 || p.nseg < 1) return WL_ERR_UNSUPPORTED;
-    const int NT = (p.M + 7) / 8;
-    if ((size_t)8 * NT * p.t_ld > (size_t)kDecodeTMaxFloats) return WL_ERR_UNSUPPORTED;
+namespace {
 
-    int blocks = 0;
-    bool any_r = false;
-    p.u_bulk = 1;
+bool aligned_to(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+// Shares `grid` CTAs out among the projections: one each, then one at a time
+// to the projection with the most blocks per CTA (never more CTAs than blocks).
+void split_ctas(DecodeArgs &p, int grid) {
+    int ncta[kMaxSeg];
+    int used = 0;
     for (int i = 0; i < p.nseg; ++i) {
-        DecodeSeg &sg = p.seg[i];
+        ncta[i] = 1;
+        ++used;
+    }
+    while (used < grid) {
+        int best = -1, best_load = 0;
+        for (int i = 0; i < p.nseg; ++i) {
+            const int nb = seg_blocks(p.seg[i]);
+            if (ncta[i] >= nb) continue;
+            const int load = (nb + ncta[i] - 1) / ncta[i];
+            if (load > best_load) {
+                best_load = load;
+                best = i;
+            }
+        }
+        if (best < 0) break;
+        ++ncta[best];
+        ++used;
+    }
+    int c = 0;
+    for (int i = 0; i < p.nseg; ++i) {
+        p.seg[i].cta_begin = c;
+        c += ncta[i];
+    }
+}
+
+}  // namespace
+
+wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
+    if (p.a.M < 1 || p.a.M > WL_DECODE_MAX_M || p.a.K < 8 || p.a.nseg < 1 || num_sms < 1) return WL_ERR_UNSUPPORTED;
+    const int NT = (p.a.M + 7) / 8;
+    if ((size_t)8 * NT * p.a.t_ld > (size_t)kDecodeTMaxFloats) return WL_ERR_UNSUPPORTED;
+
+    int blocks = 0, max_r = 0;
+    bool any_r = false, v_ok = true;
+    p.a.u_bulk = 1;
+    for (int i = 0; i < p.a.nseg; ++i) {
+        DecodeSeg &sg = p.a.seg[i];
         sg.blk_begin = blocks;
-        blocks += (sg.N + BR - 1) / BR;
+        sg.cta_begin = 0;
+        blocks += seg_blocks(sg);
         if (sg.r > 0) {
             any_r = true;
-            if (sg.r % 8 != 0 || (reinterpret_cast<uintptr_t>(sg.U) & 15u) != 0) p.u_bulk = 0;
+            max_r = sg.r > max_r ? sg.r : max_r;
+            if (sg.r % 8 != 0 || !aligned_to(sg.U, 16)) p.a.u_bulk = 0;
+            if (sg.r % 8 != 0 || !aligned_to(sg.V, 16)) v_ok = false;  // staging and ldmatrix need both
         }
     }
-    if (!any_r) p.u_bulk = 0;
-    p.total_blocks = blocks;
-    p.w3d = (p.K % CK == 0 && p.K / CK >= SC) ? 1 : 0;
+    if (!any_r) {
+        p.a.u_bulk = 0;
+        v_ok = false;
+    }
+    p.a.total_blocks = blocks;
+    const int grid = blocks < num_sms ? blocks : num_sms;
+
+    // Ring slots: each warp's share of a block's K chunks, at most four chunks.
+    const int nchunks = (p.a.K + CK - 1) / CK;
+    const int per_warp = (nchunks + NW - 1) / NW;
+    p.a.slot_chunks = per_warp < 1 ? 1 : (per_warp > kDecodeMaxSlotChunks ? kDecodeMaxSlotChunks : per_warp);
+    p.a.w3d = (p.a.K % CK == 0 && p.a.slot_chunks >= 2) ? 1 : 0;
 
     wl_status st;
-    for (int i = 0; i < p.nseg; ++i) {
-        const DecodeSeg &sg = p.seg[i];
-        if ((st = encode_map_2d(&p.tm_w[i], sg.W0, p.K, sg.N, p.K, CK, BR)) != WL_OK) return st;
-        if (p.w3d &&
-            (st = encode_map_3d(&p.tm_w3[i], sg.W0, CK, sg.N, p.K / CK, (uint64_t)p.K * 2, CK * 2, CK, BR,
-                                SC)) != WL_OK)
+    for (int i = 0; i < p.a.nseg; ++i) {
+        const DecodeSeg &sg = p.a.seg[i];
+        if ((st = encode_map_2d(&p.tm_w[i], sg.W0, p.a.K, sg.N, p.a.K, CK, BR)) != WL_OK) return st;
+        if (p.a.w3d && (st = encode_map_3d(&p.tm_w3[i], sg.W0, CK, sg.N, p.a.K / CK, (uint64_t)p.a.K * 2, CK * 2, CK,
+                                         BR, p.a.slot_chunks)) != WL_OK)
             return st;
-        if (p.u_bulk && sg.r > 0 &&
-            (st = encode_map_2d(&p.tm_u[i], sg.U, sg.r, sg.N, sg.r, CK, BR)) != WL_OK)
+        if (p.a.u_bulk && sg.r > 0 && (st = encode_map_2d(&p.tm_u[i], sg.U, sg.r, sg.N, sg.r, CK, BR)) != WL_OK)
             return st;
     }
 
-    int grid = blocks < num_sms ? blocks : num_sms;
-    if (!any_r) {
-        p.t_mode = kTNone;
-    } else {
-        // local mode when the V bytes any one CTA must read stay small
+    // T mode.  Local when the V rows any one CTA needs stay small, with the
+    // CTAs first shared out among the projections (then a CTA needs one V).
+    p.a.seg_split = 0;
+    p.a.t_mode = kTNone;
+    if (any_r) {
+        if (blocks > grid && p.a.nseg > 1) {
+            split_ctas(p.a, grid);
+            p.a.seg_split = 1;
+        }
+        p.a.t_mode = kTLocal;
         size_t worst = 0;
         for (int c = 0; c < grid; ++c) {
-            const int lo = (int)(((long long)c * blocks) / grid);
-            const int hi = (int)(((long long)(c + 1) * blocks) / grid);
+            int lo, hi;
+            cta_blocks(p.a, c, grid, lo, hi);
             size_t bytes = 0;
-            for (int i = 0; i < p.nseg; ++i) {
-                const DecodeSeg &sg = p.seg[i];
-                const int nb = (sg.N + BR - 1) / BR;
-                if (sg.r > 0 && sg.blk_begin < hi && sg.blk_begin + nb > lo) bytes += (size_t)p.K * sg.r * 2;
-            }
-            if (bytes > worst) worst = bytes;
+            for (int i = 0; i < p.a.nseg; ++i)
+                if (seg_touched(p.a.seg[i], lo, hi)) bytes += (size_t)p.a.K * p.a.seg[i].r * 2;
+            worst = bytes > worst ? bytes : worst;
         }
-        p.t_mode = worst <= kLocalVBytes ? kTLocal : kTGrid;
+        if (worst > kLocalVBytes) {
+            p.a.t_mode = kTGrid;
+            p.a.seg_split = 0;
+        }
     }
-    // Stage x in shared memory when it fits next to the ring.
-    p.x_ld = p.K + 8;
-    const uint32_t x_bytes = (uint32_t)p.M * p.x_ld * 2;
-    p.x_smem = smem_layout(NT, p.t_ld, x_bytes).total <= kDecodeMaxSmem ? 1 : 0;
+    int min_blocks = blocks, max_blocks = 0;
+    size_t v_bytes = 0;
+    for (int c = 0; c < grid; ++c) {
+        int lo, hi;
+        cta_blocks(p.a, c, grid, lo, hi);
+        min_blocks = hi - lo < min_blocks ? hi - lo : min_blocks;
+        max_blocks = hi - lo > max_blocks ? hi - lo : max_blocks;
+        size_t bytes = 0;
+        for (int i = 0; i < p.a.nseg; ++i) {
+            int k0, k1;
+            v_range(p.a, i, c, grid, lo, hi, k0, k1);
+            bytes += (size_t)(k1 - k0) * p.a.seg[i].r * 2;
+        }
+        v_bytes = bytes > v_bytes ? bytes : v_bytes;
+    }
+    p.a.lag = p.a.t_mode == kTGrid ? (min_blocks < kDecodeMaxLag ? (min_blocks < 1 ? 1 : min_blocks) : kDecodeMaxLag) : 0;
+    p.a.x_ld = p.a.K + 8;
+
+    // Shared memory: the compact variant (two CTAs per SM) for calls whose
+    // per-CTA stream is short, when x fits beside a one-slot ring; otherwise
+    // the full-size one.  Within the budget: x, then the staged V rows, then
+    // more ring slots (up to 192 KB of ring).
+    const size_t cta_bytes = (size_t)max_blocks * BR * ((size_t)p.a.K + (size_t)max_r) * 2;
+    bool done = false;
+    for (int pass = 0; pass < 2 && !done; ++pass) {
+        const bool small = pass == 0;
+        if (small && cta_bytes > kSmallCtaBytes) continue;
+        const uint32_t budget = small ? kSmallSmem : kDecodeMaxSmem;
+        p.a.slots = 1;
+        p.a.x_smem = 1;
+        p.a.v_stage = 0;
+        p.a.v_bytes = 0;
+        if (smem_layout(p.a, NT).total > budget) {
+            if (small) continue;
+            p.a.x_smem = 0;
+        }
+        if (v_ok && v_bytes > 0) {
+            // the staged rows plus room for the rows past the last one that a
+            // 16-row k-step reads (and masks)
+            p.a.v_stage = 1;
+            p.a.v_bytes = (int)(v_bytes + 16 * (size_t)max_r * 2);
+            if (smem_layout(p.a, NT).total > budget) {
+                p.a.v_stage = 0;
+                p.a.v_bytes = 0;
+            }
+        }
+        while (p.a.slots < kDecodeMaxSlots) {
+            ++p.a.slots;
+            const SmemLayout Lg = smem_layout(p.a, NT);
+            if (Lg.total > budget || Lg.ring_bytes > kMaxRingBytes) {
+                --p.a.slots;
+                break;
+            }
+        }
+        if (smem_layout(p.a, NT).total > budget) return WL_ERR_UNSUPPORTED;
+        plan->small = small ? 1 : 0;
+        done = true;
+    }
+    if (!done) return WL_ERR_UNSUPPORTED;
     plan->grid = grid;
-    plan->smem = smem_layout(NT, p.t_ld, p.x_smem ? x_bytes : 0u).total;
-    plan->tpart_bytes = p.t_mode == kTGrid ? (size_t)(grid + 1) * p.M * p.t_ld * sizeof(float) : 0;
+    plan->smem = smem_layout(p.a, NT).total;
+    plan->tpart_bytes = p.a.t_mode == kTGrid ? (size_t)(grid + 1) * p.a.M * p.a.t_ld * sizeof(float) : 0;
     return WL_OK;
 }
 
-template <int NT, bool XS>
-static cudaError_t launch_decode_nt(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
-    // Opt in to the large shared-memory carve-out once per device.
+template <int NT, bool XS, bool SMALL>
+static cudaError_t launch_decode_v(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+    // Opt in to the large shared-memory carve-out once per device: both
+    // variants run with all of the SM's shared memory configured, so the
+    // compact one can hold two CTAs (of consecutive calls) per SM.
     static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        e = cudaFuncSetAttribute(decode_kernel<NT, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kDecodeMaxSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.grid);
-    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -859,14 +1219,20 @@ static cudaError_t launch_decode_nt(const DecodeParams &p, const DecodePlan &pla
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<NT, XS>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<NT, XS, SMALL>, p);
+}
+
+template <int NT>
+static cudaError_t launch_decode_nt(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+    if (plan.small)  // the planner takes the compact variant only with x in shared memory
+        return p.a.x_smem ? launch_decode_v<NT, true, true>(p, plan, stream) : cudaErrorInvalidValue;
+    return p.a.x_smem ? launch_decode_v<NT, true, false>(p, plan, stream)
+                    : launch_decode_v<NT, false, false>(p, plan, stream);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
-    if (p.M <= 8)
-        return p.x_smem ? launch_decode_nt<1, true>(p, plan, stream) : launch_decode_nt<1, false>(p, plan, stream);
-    if (p.M <= 16)
-        return p.x_smem ? launch_decode_nt<2, true>(p, plan, stream) : launch_decode_nt<2, false>(p, plan, stream);
+    if (p.a.M <= 8) return launch_decode_nt<1>(p, plan, stream);
+    if (p.a.M <= 16) return launch_decode_nt<2>(p, plan, stream);
     return cudaErrorInvalidValue;
 }
 

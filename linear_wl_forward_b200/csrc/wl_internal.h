@@ -14,17 +14,16 @@ constexpr int kMaxSeg = WL_MAX_PROJ;
 
 // --------------------------------------------------------------- decode ----
 // Streaming decode kernel: M <= WL_DECODE_MAX_M tokens.  The projections of a
-// stacked call are concatenated into one row space [0, total_rows).
-constexpr int kDecodeWarps = 8;          // consumer warps
-constexpr int kDecodeConsumers = 32 * kDecodeWarps;
-constexpr int kDecodeThreads = kDecodeConsumers;  // every warp feeds its own ring
-constexpr int kDecodeBlockRows = 16;     // rows of one MMA row block
-constexpr int kDecodeChunkK = 64;        // K columns per TMA box (128 B, swizzled)
+// stacked call are concatenated into one list of 16-row blocks.
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodeThreads = 32 * kDecodeWarps;
+constexpr int kDecodeBlockRows = 16;      // rows of one MMA row block
+constexpr int kDecodeChunkK = 64;         // K columns per TMA box (128 B, swizzled)
 constexpr int kDecodeChunkBytes = kDecodeBlockRows * kDecodeChunkK * 2;  // 2 KB
-constexpr int kDecodeSlotChunks = 2;     // chunks per ring slot: 16 rows x 128 columns
-constexpr int kDecodeSlotBytes = kDecodeSlotChunks * kDecodeChunkBytes;  // 4 KB
-constexpr int kDecodeSlotsPerWarp = 4;
-constexpr int kDecodeTMaxFloats = 12288; // M (rounded up to 8) * (sum of ranks) in shared memory
+constexpr int kDecodeMaxSlotChunks = 4;   // a ring slot holds up to 16 rows x 256 columns
+constexpr int kDecodeMaxSlots = 4;        // ring slots per warp
+constexpr int kDecodeTMaxFloats = 12288;  // M (rounded up to 8) * (sum of ranks) in shared memory
+constexpr int kDecodeMaxLag = 2;          // blocks by which the U part of a block may trail its W0 part
 
 // How a CTA obtains T = V^T x.
 enum DecodeTMode : int {
@@ -44,39 +43,55 @@ struct DecodeSeg {
     int r;
     int t_off;      // column offset of this projection's T slice
     int blk_begin;  // first 16-row block of this projection in the call's block list
+    int cta_begin;  // seg_split: first CTA of this projection
 };
 
-struct DecodeParams {
-    CUtensorMap tm_w[kMaxSeg];   // W0: 2-D {K, N}, box {64, 16}, 128-B swizzle
-    CUtensorMap tm_w3[kMaxSeg];  // W0: 3-D {64, N, K/64}, box {64, 16, 4} (when w3d)
-    CUtensorMap tm_u[kMaxSeg];   // U:  2-D {r, N}, box {64, 16} (when u_bulk)
+// Everything the decode kernel reads except the tensor maps.  The kernel
+// copies it into shared memory once at the start: a parameter block is new
+// for every launch, so reading it in place costs a chain of constant-cache
+// misses right on the path after the wait for the previous kernel.
+struct DecodeArgs {
     DecodeSeg seg[kMaxSeg];
     int nseg;
     int M, K;
     int total_blocks;
-    int t_ld;       // row stride of T (sum of ranks)
-    int w3d;        // K % 64 == 0: a full slot of W0 is one 3-D box
-    int u_bulk;     // every U is TMA-able (r % 8 == 0, 16-byte aligned)
-    int t_mode;     // DecodeTMode
-    int x_smem;     // x is staged in shared memory (rows padded to x_ld elements)
+    int seg_split;    // CTAs are split over the projections in proportion to their blocks
+    int t_ld;         // row stride of T (sum of ranks)
+    int slot_chunks;  // 64-column chunks per ring slot (1 .. kDecodeMaxSlotChunks)
+    int slots;        // ring slots per warp (1 .. kDecodeMaxSlots)
+    int w3d;          // K % 64 == 0 and slot_chunks > 1: a full W0 slot is one 3-D box
+    int u_bulk;       // every U is TMA-able (r % 8 == 0, 16-byte aligned)
+    int t_mode;       // DecodeTMode
+    int lag;          // kTGrid: the U part of block b runs in step b + lag
+    int x_smem;       // x is staged in shared memory (rows padded to x_ld elements)
     int x_ld;
+    int v_stage;      // each CTA bulk-copies the V rows it needs for T into shared memory
+    int v_bytes;      // shared memory reserved for them (largest over the CTAs)
     const __nv_bfloat16 *x;
-    float *Tpart;   // kTGrid: [grid][M][t_ld] partial sums, then [M][t_ld] final T
+    float *Tpart;     // kTGrid: [grid][M][t_ld] partial sums, then [M][t_ld] final T
     unsigned int *sync;  // kTGrid: [0], [1] arrival counts, [2] departures; self-resetting
     int *status;
     unsigned long long timeout_ns;
 };
 
+struct DecodeParams {
+    DecodeArgs a;
+    CUtensorMap tm_w[kMaxSeg];   // W0: 2-D {K, N}, box {64, 16}, 128-B swizzle
+    CUtensorMap tm_w3[kMaxSeg];  // W0: 3-D {64, N, K/64}, box {64, 16, slot_chunks} (when w3d)
+    CUtensorMap tm_u[kMaxSeg];   // U:  2-D {r, N}, box {64, 16} (when u_bulk)
+};
+
 // Host-side planning shared by every decode entry point.
 struct DecodePlan {
     int grid;
+    int small;           // the compact variant, two CTAs per SM (consecutive calls overlap)
     size_t smem;
     size_t tpart_bytes;  // scratch for kTGrid partial sums and final T (0 otherwise)
 };
-// Fills the block list, the tensor maps, p.w3d, p.u_bulk and p.t_mode; returns
-// WL_ERR_UNSUPPORTED if the shape cannot take the decode path (M above
-// WL_DECODE_MAX_M, or M rounded up to 8 times the sum of ranks above
-// kDecodeTMaxFloats).
+// Fills the block list, the CTA split, the tensor maps and the ring, T and
+// shared-memory choices; returns WL_ERR_UNSUPPORTED if the shape cannot take
+// the decode path (M above WL_DECODE_MAX_M, or M rounded up to 8 times the sum
+// of ranks above kDecodeTMaxFloats).
 wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan);
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
 

@@ -95,7 +95,7 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
 
     static DecodeParams dp;  // large (tensor maps); guarded by g_noalloc_mu
     std::memset(&dp, 0, sizeof dp);
-    DecodeSeg &sg = dp.seg[0];
+    DecodeSeg &sg = dp.a.seg[0];
     sg.W0 = reinterpret_cast<const __nv_bfloat16 *>(W0);
     sg.s = s;
     sg.U = reinterpret_cast<const __nv_bfloat16 *>(U);
@@ -104,12 +104,12 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
     sg.N = N;
     sg.r = r;
     sg.t_off = 0;
-    dp.nseg = 1;
-    dp.M = M;
-    dp.K = K;
-    dp.t_ld = r;
-    dp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-    dp.timeout_ns = 2000000000ull;
+    dp.a.nseg = 1;
+    dp.a.M = M;
+    dp.a.K = K;
+    dp.a.t_ld = r;
+    dp.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    dp.a.timeout_ns = 2000000000ull;
     DecodePlan plan;
     if ((st = plan_decode(dp, d->num_sms, &plan)) != WL_OK) return st;
     // Scratch: the word block, then the partial sums of V^T x ((grid+1) x M x r fp32).
@@ -119,8 +119,8 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
     // arrival counters, which must start at zero, on the caller's stream.
     if (cudaMemsetAsync(d->scratch, 0, kWordsBytes, stream) != cudaSuccess) return WL_ERR_CUDA;
     int *words = reinterpret_cast<int *>(d->scratch);
-    dp.status = words;
-    dp.sync = reinterpret_cast<unsigned int *>(words + 8);
-    dp.Tpart = reinterpret_cast<float *>(d->scratch + kWordsBytes);
+    dp.a.status = words;
+    dp.a.sync = reinterpret_cast<unsigned int *>(words + 8);
+    dp.a.Tpart = reinterpret_cast<float *>(d->scratch + kWordsBytes);
     return launch_decode(dp, plan, stream) == cudaSuccess ? WL_OK : WL_ERR_CUDA;
 }
