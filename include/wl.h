@@ -95,7 +95,13 @@ typedef enum {
  *   V  : device, K x r bf16 row-major (NULL iff r == 0)
  *   y  : device, M x N bf16 row-major (written)
  * M, N >= 0 (0 is a no-op), K >= 0 with K % 8 == 0 (K == 0 writes y = 0),
- * 0 <= r <= WL_MAX_RANK.  Asynchronous on `stream` (cudaStream_t). */
+ * 0 <= r <= WL_MAX_RANK.  Asynchronous on `stream` (cudaStream_t).
+ * Ordering: the decode kernel is launched with programmatic dependent launch
+ * and starts streaming W0, U, V and s while the previous kernel in the stream
+ * still runs (x, y and the scratch are touched only after that kernel has
+ * finished).  So W0, s, U and V must not be the outputs of the immediately
+ * preceding forward call of this library on the same stream; outputs of any
+ * other kernel are safe. */
 wl_status wl_linear_forward(const wl_bf16 *x, const wl_bf16 *W0, const float *s,
                             const wl_bf16 *U, const wl_bf16 *V, wl_bf16 *y,
                             int M, int N, int K, int r, void *stream);
