@@ -321,6 +321,24 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank takes part in the all-reduce (NCCL
+    on the GPU, gloo on the host in the tests)."""
+    if world <= 1:
+        return ms
+    import torch.distributed as dist
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(world, bytes_per_step, steps, ms_total):
+    """Whole-job GB/s: every replica streams the same bytes; the job takes as
+    long as its slowest rank."""
+    return world * bytes_per_step * steps / (ms_total * 1e-3) / 1e9
+
+
 def run_reference(args):
     world, rank, _ = dist_setup()
     if rank != 0:
@@ -409,14 +427,10 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms_total = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms_total], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), world, "cuda")
     status = wl.last_device_status()
     ms_step = ms_total / args.steps
-    value = world * wbytes * args.steps / (ms_total * 1e-3) / 1e9
+    value = replica_value(world, wbytes, args.steps, ms_total)
 
     # e2e: eager public API calls, x H2D from pinned memory, all y D2H, per step
     xs_host = {}
@@ -448,12 +462,9 @@ def main():
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * wbytes / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3) / e2e_steps,
+                            world, "cuda")
+    e2e_value = replica_value(world, wbytes, 1, e2e_ms)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
