@@ -217,12 +217,20 @@ def time_graph(g, reps):
 
 
 # --------------------------------------------------------------- roofline --
-def decode_roofline(wl, peaks):
-    """Dominant kernel of the Gemma-3-1B decode step: the stacked gate/up
-    decode call (2 x 4096 x 1152, rank 16, M = 1).  Timed alone with CUDA
-    events over a graph of calls that rotate through enough distinct bundles
-    (> 3x L2) that every launch streams its weights from HBM."""
-    N, K, r, M = 4096, 1152, 16, 1
+ROOFLINE_CALLS = {
+    # name: (N per projection, K, r, M, label)
+    "gemma3_gate_up": (4096, 1152, 16, 1, "stacked gate/up decode, 2 x 4096 x 1152, r=16, M=1"),
+    "gemma4_gate_up": (21504, 5376, 256, 1, "stacked gate/up decode, 2 x 21504 x 5376, r=256, M=1"),
+    "gemma4_gate_up_m16": (21504, 5376, 256, 16, "stacked gate/up decode, 2 x 21504 x 5376, r=256, M=16"),
+}
+
+
+def decode_roofline(wl, peaks, call="gemma3_gate_up"):
+    """One stacked decode call timed alone with CUDA events over a graph of
+    calls that rotate through enough distinct bundles (> 3x L2) that every
+    launch streams its weights from HBM.  The default is the dominant kernel
+    of the Gemma-3-1B decode step: the stacked gate/up call."""
+    N, K, r, M, label = ROOFLINE_CALLS[call]
     per_call = 2 * footprint.call_weight_bytes(N, K, r) + footprint.call_io_bytes(M, 2 * N, K)
     copies = max(4, (3 * L2_BYTES) // (2 * N * K * 2) + 1)
     calls = []
@@ -235,23 +243,24 @@ def decode_roofline(wl, peaks):
     g = capture(step, 3)
     ms = time_graph(g, 20) / copies
     achieved = per_call / (ms * 1e-3) / 1e9
-    traffic = traffic_from_profile("decode_kernel")
+    traffic = traffic_from_profile("decode_kernel", call)
     return {"kernel": "decode_kernel (one launch per call: W0 x, V^T x and the epilogue fused)",
-            "call": "stacked gate/up decode, 2 x 4096 x 1152, r=16, M=1",
+            "call": label,
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic, "algorithmic_bytes": per_call, "us_per_launch": round(ms * 1e3, 3),
             "peak_source": peaks["source"]}
 
 
-def traffic_from_profile(kernel):
-    """DRAM bytes per launch from the committed ncu summary, only while the
-    kernel source is unchanged since the counters were taken."""
+def traffic_from_profile(kernel, call):
+    """DRAM bytes per launch of `kernel` on `call` from the committed ncu
+    summary, only while the kernel source is unchanged since the counters
+    were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f).get(kernel)
+        rec = json.load(f).get(f"{kernel}/{call}")
     if not rec:
         return None
     src = os.path.join(ROOT, "linear_wl_forward_b200", "csrc", rec["source"])
@@ -376,6 +385,8 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--roofline-only", action="store_true",
                     help="time only the dominant kernel's call (the command the ncu summaries profile)")
+    ap.add_argument("--call", default="gemma3_gate_up", choices=sorted(ROOFLINE_CALLS),
+                    help="the call --roofline-only times")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -399,7 +410,7 @@ def main():
     wl.lib()  # fails loudly if the CUDA library is missing
     peaks = load_peaks()
     if args.roofline_only:
-        print(json.dumps({"roofline": decode_roofline(wl, peaks)}), flush=True)
+        print(json.dumps({"roofline": decode_roofline(wl, peaks, args.call)}), flush=True)
         return
 
     calls, wbytes, flops, desc = build_workload(args.workload)

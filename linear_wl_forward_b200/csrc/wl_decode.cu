@@ -39,10 +39,12 @@
 //    the warps splitting the k-steps (CUDA cores when V cannot be staged);
 //  * grid: otherwise each CTA forms partial sums over a 1/grid slice of K for
 //    every projection (the warps splitting the 16-column tiles of r) and
-//    writes them to scratch (phase A); one step later it
-//    waits for all CTAs' partials and adds up its 1/grid share of the outputs
-//    over all CTAs (phase B); `lag` steps in it waits for all shares and loads
-//    the slices it needs (phase C).  Meanwhile the W0 stream runs on: in step
+//    writes them to scratch (phase A); then it waits for all CTAs' partials
+//    and adds up its 1/grid share of the outputs over all CTAs (phase B);
+//    then it waits for all shares and loads the slices it needs (phase C, in
+//    step `lag`).  The steps of the three phases depend on the CTA's block
+//    count (the chain starts at once for a CTA with few blocks).
+//    Meanwhile the W0 stream runs on: in step
 //    t a CTA does the W0 part of its block t and the U part of block t - lag,
 //    keeping z = W0 x of the blocks in between in shared memory.  The counters
 //    reset themselves once every CTA is past both counts.
@@ -674,11 +676,11 @@ __host__ __device__ inline SmemLayout smem_layout(const DecodeArgs &p, int NT) {
     L.xs_off = L.red_off + (epi_red > vtx_red ? epi_red : vtx_red);
     const uint32_t x_bytes = p.x_smem ? (uint32_t)p.M * p.x_ld * 2u : 0u;
     L.vs_off = L.xs_off + ((x_bytes + 127u) & ~127u);
-    const uint32_t v_bytes = p.v_stage ? (uint32_t)p.v_bytes : 0u;
+    const uint32_t v_bytes = (p.v_stage && !p.v_in_ring) ? (uint32_t)p.v_bytes : 0u;
     L.zs_off = L.vs_off + ((v_bytes + 127u) & ~127u);
     const uint32_t z_bytes = p.lag > 0 ? (uint32_t)(p.lag + 1) * BR * p.M * 4u : 0u;
     L.bar_off = L.zs_off + ((z_bytes + 127u) & ~127u);
-    L.flag_off = L.bar_off + (uint32_t)(NW * p.slots + 1) * 8u;
+    L.flag_off = L.bar_off + (uint32_t)(NW * p.slots + 5) * 8u;
     L.total = L.flag_off + 16u + 1024u + kArgsBytes;  // + the copy of the arguments, before the ring
     return L;
 }
@@ -701,16 +703,17 @@ __device__ __forceinline__ Step step_info(const DecodeArgs &p, int blk_lo, int n
     return S;
 }
 
-// The scales this thread applies in step t: for y of block t (written in
-// this step when it has no delta or lag is 0) and of block t - lag.
-__device__ __forceinline__ void step_scales(const DecodeArgs &p, const Step &S, int tid, float &sc_w,
+// The scales for output index o of step t's epilogue: for y of block t
+// (written then when it has no delta or lag is 0) and of block t - lag.
+__device__ __forceinline__ void step_scales(const DecodeArgs &p, const Step &S, int o, float &sc_w,
                                             float &sc_u) {
     const int M = p.M;
     sc_w = sc_u = 0.f;
-    if (S.has_w && (S.rw == 0 || p.lag == 0) && tid < S.bw.nrows * M)
-        sc_w = __ldg(p.seg[S.bw.sp].s + S.bw.row0 + tid / M);
-    if (S.has_u && S.ru > 0 && p.lag > 0 && tid < S.bu.nrows * M)
-        sc_u = __ldg(p.seg[S.bu.sp].s + S.bu.row0 + tid / M);
+    if (o < 0) return;
+    if (S.has_w && (S.rw == 0 || p.lag == 0) && o < S.bw.nrows * M)
+        sc_w = __ldg(p.seg[S.bw.sp].s + S.bw.row0 + o / M);
+    if (S.has_u && S.ru > 0 && p.lag > 0 && o < S.bu.nrows * M)
+        sc_u = __ldg(p.seg[S.bu.sp].s + S.bu.row0 + o / M);
 }
 
 }  // namespace
@@ -731,6 +734,32 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     }
     __syncthreads();
     const DecodeArgs &p = *reinterpret_cast<const DecodeArgs *>(smem_raw);
+    int blk_lo, blk_hi;
+    cta_blocks(p, blockIdx.x, gridDim.x, blk_lo, blk_hi);
+    const int nblk = blk_hi - blk_lo;
+    // Grid-mode T schedule of this CTA: phase A (partial sums) in step t_a,
+    // phase B (the reduction) in step t_b, phase C (T loaded) in step lag,
+    // which is where the first U part runs.  With few blocks there is little
+    // W0 to overlap, so the chain starts at once; with many, phase A waits
+    // for the first step's W0 part (the stream is under way) unless V holds
+    // a ring level, whose copies stop until phase A is done.
+    int t_a = 0, t_b = 0;
+    if (p.t_mode == kTGrid) {
+        int lag;
+        if (nblk <= 1) {
+            lag = 1;
+        } else if (nblk <= 3 || p.v_in_ring) {
+            t_b = 1;
+            lag = 2;
+        } else {
+            t_a = 1;
+            t_b = 2;
+            lag = 3;
+        }
+        __syncthreads();  // every thread has read the copied arguments
+        if (threadIdx.x == 0) reinterpret_cast<DecodeArgs *>(smem_raw)->lag = lag;
+        __syncthreads();
+    }
     const uint32_t raw_addr = smem_addr(smem_raw) + kArgsBytes;
     uint8_t *smem = smem_raw + kArgsBytes + ((1024u - (raw_addr & 1023u)) & 1023u);
     const SmemLayout L = smem_layout(p, NT);
@@ -738,21 +767,27 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     float *Ts = reinterpret_cast<float *>(smem + L.ts_off);    // [M][t_ld]
     float *red = reinterpret_cast<float *>(smem + L.red_off);  // step sums; T scratch before the steps
     __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(smem + L.xs_off);  // [M][x_ld]
-    uint8_t *vs = smem + L.vs_off;                             // staged V rows
     float *zs = reinterpret_cast<float *>(smem + L.zs_off);    // [lag + 1][16 * M]: z awaiting U T
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);  // [NW][slots]
     const int SLOTS = p.slots;
     uint64_t *vbar = full + NW * SLOTS;  // V rows staged
+    uint64_t *red_full = vbar + 1;       // [2] every warp's sums of a step are in
+    uint64_t *red_empty = vbar + 3;      // [2] the step's epilogue has read them
+    // staged V rows: their own region, or the ring's last slot level (handed
+    // to the W0 stream once T's sums are formed)
+    uint8_t *vs = p.v_in_ring ? smem + (size_t)(SLOTS - 1) * NW * L.slot_bytes : smem + L.vs_off;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.flag_off);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-    int blk_lo, blk_hi;
-    cta_blocks(p, blockIdx.x, gridDim.x, blk_lo, blk_hi);
-    const int nblk = blk_hi - blk_lo, nsteps = nblk + p.lag;
+    const int nsteps = nblk + p.lag;
     const int K = p.K, M = p.M, SC = p.slot_chunks;
 
     if (tid == 0) {
         for (int i = 0; i < NW * SLOTS + 1; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&red_full[i], NW);
+            mbar_init(&red_empty[i], (BR * p.M + 31) / 32);
+        }
         *abort_flag = 0;
         fence_barrier_init();
         for (int i = 0; i < p.nseg; ++i) {
@@ -771,8 +806,11 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     // Each warp feeds its own ring; W0, U, V and s are parameters, so the V
     // rows for T and the whole ring are requested before waiting for the
     // previous kernel.
+    // Slot s of warp w is at ring + (s * NW + w) * slot_bytes (slot-major, so
+    // one slot level is contiguous).
     uint64_t *my_full = full + warp * SLOTS;
-    uint8_t *my_ring = ring + (size_t)warp * SLOTS * L.slot_bytes;
+    uint8_t *my_ring = ring + (size_t)warp * L.slot_bytes;
+    const uint32_t level_bytes = (uint32_t)NW * L.slot_bytes;
     const uint64_t pol = stream_policy();
     WarpSeq iq;  // issue position
     bool more = seq_first(p, warp, w0_slots, blk_lo, nblk, iq);
@@ -780,7 +818,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     int isl = 0;  // ring slot of the next copy
     auto issue_next = [&]() {
         if (lane == 0)
-            issue_slot(P, p, iq, w0_lo, w0_hi, my_ring + (size_t)isl * L.slot_bytes, &my_full[isl], pol);
+            issue_slot(P, p, iq, w0_lo, w0_hi, my_ring + (size_t)isl * level_bytes, &my_full[isl], pol);
         ++issued;
         if (++isl == SLOTS) isl = 0;
         more = seq_next(p, warp, w0_slots, blk_lo, nblk, iq);
@@ -802,10 +840,18 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             off += bytes;
         }
     }
-    while (more && issued < (uint32_t)SLOTS) issue_next();
+    // the whole ring, less the level that holds V until T's sums are formed
+    const uint32_t pre_slots = p.v_in_ring ? (uint32_t)SLOTS - 1u : (uint32_t)SLOTS;
+    while (more && issued < pre_slots) issue_next();
+    // Output index of this thread in the epilogue of step u (-1: not its turn).
+    const int E = (BR * M + 31) / 32;  // warps per epilogue
+    auto epi_out = [&](int u) -> int {
+        const int rel = (warp - (u * E) % NW + NW) % NW;
+        return rel < E ? rel * 32 + lane : -1;
+    };
     Step S = step_info(p, blk_lo, nblk, 0);
     float sc_w, sc_u;
-    step_scales(p, S, tid, sc_w, sc_u);
+    step_scales(p, S, epi_out(0), sc_w, sc_u);
 
     pdl_wait_primary();  // the previous kernel is done: x and the scratch are ours
     const __nv_bfloat16 *xsrc = p.x;
@@ -828,8 +874,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     if (p.t_mode != kTNone && p.v_stage)
         ok = !__syncthreads_or(!mbar_wait(vbar, 0, p.status, p.timeout_ns) || *abort_flag != 0);
     if (ok && p.t_mode == kTLocal) form_t_local<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red, Ts);
-    if (ok && p.t_mode == kTGrid) grid_t_partials<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red);
-    const int t_reduce = p.lag >= 2 ? 1 : 0;  // grid mode: step of phase B (phase C is at step lag)
+
 
     const int g = lane >> 2, q = lane & 3;          // fragment row / column-pair index
     const int lrow = lane & 15, lhalf = lane >> 4;  // ldmatrix source row / k half
@@ -853,6 +898,9 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     uint32_t consumed = 0;
     int csl = 0;       // ring slot of the next copy to consume
     uint32_t cph = 0;  // its barrier phase parity
+    // While the ring's last level holds V, the copies (which take the slots in
+    // rotation) stop before it.
+    bool v_held = p.v_in_ring != 0;
     // Consumed the slot: every lane's fragments were used by the MMAs above;
     // order those generic-proxy reads before the async-proxy refill.
     auto release_slot = [&]() {
@@ -862,16 +910,73 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             cph ^= 1u;
         }
         __syncwarp();
-        if (more) {
+        if (more && !v_held) {
             if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             issue_next();
         }
     };
+    // Once every thread is past its reads of V (the T routines end with a
+    // barrier), the level that held V goes back to the W0 stream and the ring
+    // is topped up.
+    auto release_v_level = [&]() {
+        v_held = false;
+        if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        while (more && issued < consumed + (uint32_t)SLOTS) issue_next();
+    };
+    if (p.v_in_ring && p.t_mode == kTLocal) release_v_level();
 
-    int buf = 0;
+    // Epilogue of step u: the warp's share of y for the blocks of step u (or
+    // z kept for a later U part), from all warps' sums in buffer u & 1.  It
+    // is done by E consecutive warps starting at (u * E) % NW, so the work
+    // rotates over the warps; wait_full: wait for all warps' sums first.
+    auto epilogue = [&](int u, const Step &Su, float su_w, float su_u, bool wait_full) -> bool {
+        const int o = epi_out(u);
+        if (o < 0) return true;
+        const int b = u & 1;
+        if (wait_full && !warp_wait(&red_full[b], (uint32_t)(u >> 1) & 1u, p, abort_flag)) return false;
+        const float *rbu = red + (size_t)b * NW * 32 * 8 * NT;
+        if (o < BR * M) {
+            const int row = o / M, n = o - row * M;
+            const int nt = n >> 3, tc = n & 7;
+            const int fl = (row & 7) * 4 + (tc >> 1);  // fragment lane
+            const int fe = (row >> 3) * 2 + (tc & 1);   // element in that lane
+            float z = 0.f, d = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float *f = rbu + ((size_t)(w * 32 + fl) * NT + nt) * 8;
+                z += f[fe];
+                d += f[4 + fe];
+            }
+            if (Su.has_w && row < Su.bw.nrows) {
+                const DecodeSeg &sg = p.seg[Su.bw.sp];
+                if (Su.rw > 0 && p.lag > 0)
+                    zs[(u % (p.lag + 1)) * BR * M + o] = z;  // y once U T of the block is in
+                else
+                    sg.y[(size_t)n * sg.N + Su.bw.row0 + row] =
+                        __float2bfloat16_rn(fmaf(su_w, z, p.lag == 0 ? d : 0.f));
+            }
+            if (Su.has_u && Su.ru > 0 && p.lag > 0 && row < Su.bu.nrows) {
+                const DecodeSeg &sg = p.seg[Su.bu.sp];
+                const float zu = zs[((u - p.lag) % (p.lag + 1)) * BR * M + o];
+                sg.y[(size_t)n * sg.N + Su.bu.row0 + row] = __float2bfloat16_rn(fmaf(su_u, zu, d));
+            }
+        }
+        if (!SMALL) {  // the compact variant's steps all end with a CTA barrier
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[b]);
+        }
+        return true;
+    };
+    int pend = -1;  // step whose epilogue is still due
+    float scp_w = 0.f, scp_u = 0.f;
     for (int t = 0; t < nsteps && ok; ++t) {
         if (p.t_mode == kTGrid) {
-            if (t == t_reduce) ok = grid_t_reduce(p, abort_flag);
+            if (t == t_a) {
+                grid_t_partials<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red);
+                if (p.v_in_ring) release_v_level();
+            }
+            if (t == t_b) ok = grid_t_reduce(p, abort_flag);
             if (ok && t == p.lag) ok = grid_t_load(p, blk_lo, blk_hi, Ts, abort_flag);
             if (!ok) break;
         }
@@ -887,7 +992,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
                 ok = false;  // the warps decide together at the step barrier
                 break;
             }
-            const uint32_t sbase = ring_s + (uint32_t)csl * L.slot_bytes;
+            const uint32_t sbase = ring_s + (uint32_t)csl * level_bytes;
             const int c_lo = w0_lo + s * SC;
             const int nch = min(SC, w0_hi - c_lo);
             for (int cc = 0; cc < nch; ++cc) {
@@ -913,7 +1018,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
                     ok = false;
                     break;
                 }
-                const uint32_t sbase = ring_s + (uint32_t)csl * L.slot_bytes;
+                const uint32_t sbase = ring_s + (uint32_t)csl * level_bytes;
                 const int c_lo = u_lo + s * SC;
                 const int nch = min(SC, u_hi - c_lo);
                 for (int cc = 0; cc < nch; ++cc)
@@ -958,54 +1063,57 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             }
         }
 
-        // ---- add the eight warps' accumulators ----
-        float *rb = red + (size_t)buf * NW * 32 * 8 * NT;
+        // ---- publish this warp's sums of step t ----
+        const int rbuf = t & 1;
+        float *rb = red + (size_t)rbuf * NW * 32 * 8 * NT;
+        // the buffer is free once the epilogue of step t - 2 has read it
+        if (!SMALL && ok && t >= 2)
+            ok = warp_wait(&red_empty[rbuf], (uint32_t)((t - 2) >> 1) & 1u, p, abort_flag);
+        if (ok) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float4 *dst = reinterpret_cast<float4 *>(rb + ((size_t)(warp * 32 + lane) * NT + nt) * 8);
-            dst[0] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
-            dst[1] = make_float4(acu[nt][0], acu[nt][1], acu[nt][2], acu[nt][3]);
+            for (int nt = 0; nt < NT; ++nt) {
+                float4 *dst = reinterpret_cast<float4 *>(rb + ((size_t)(warp * 32 + lane) * NT + nt) * 8);
+                dst[0] = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+                dst[1] = make_float4(acu[nt][0], acu[nt][1], acu[nt][2], acu[nt][3]);
+            }
+            if (!SMALL) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&red_full[rbuf]);
+            }
         }
-        if (__syncthreads_or(!ok || *abort_flag != 0)) {
-            ok = false;  // every warp leaves together
+        // Steps of a short call, and steps that carry grid-mode T phases (the
+        // phases need every warp), end with a CTA barrier and their epilogue;
+        // elsewhere no warp waits for the others except through the two
+        // buffers, and the epilogue runs one step behind.
+        const bool sync_step = SMALL || (p.t_mode == kTGrid && t <= p.lag);
+        if (sync_step) {
+            if (__syncthreads_or(!ok || *abort_flag != 0)) {
+                ok = false;  // every warp leaves together
+                break;
+            }
+        } else if (!ok) {
             break;
         }
         const Step cur = S;
         const float cur_sc_w = sc_w, cur_sc_u = sc_u;
         if (t + 1 < nsteps) {
             // the next step's blocks and scales, loaded now so their latency
-            // hides behind this step's epilogue and the next step's MMAs
+            // hides behind the next step's MMAs
             S = step_info(p, blk_lo, nblk, t + 1);
-            step_scales(p, S, tid, sc_w, sc_u);
+            step_scales(p, S, epi_out(t + 1), sc_w, sc_u);
         }
-        if (tid < BR * M) {  // 16 * M <= the thread count
-            const int row = tid / M, n = tid - row * M;
-            const int nt = n >> 3, tc = n & 7;
-            const int fl = (row & 7) * 4 + (tc >> 1);  // fragment lane
-            const int fe = (row >> 3) * 2 + (tc & 1);   // element in that lane
-            float z = 0.f, d = 0.f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float *f = rb + ((size_t)(w * 32 + fl) * NT + nt) * 8;
-                z += f[fe];
-                d += f[4 + fe];
-            }
-            if (cur.has_w && row < cur.bw.nrows) {
-                const DecodeSeg &sg = p.seg[cur.bw.sp];
-                if (cur.rw > 0 && p.lag > 0)
-                    zs[(t % (p.lag + 1)) * BR * M + tid] = z;  // y once U T of the block is in
-                else
-                    sg.y[(size_t)n * sg.N + cur.bw.row0 + row] =
-                        __float2bfloat16_rn(fmaf(cur_sc_w, z, p.lag == 0 ? d : 0.f));
-            }
-            if (cur.has_u && cur.ru > 0 && p.lag > 0 && row < cur.bu.nrows) {
-                const DecodeSeg &sg = p.seg[cur.bu.sp];
-                const float zu = zs[((t - p.lag) % (p.lag + 1)) * BR * M + tid];
-                sg.y[(size_t)n * sg.N + cur.bu.row0 + row] = __float2bfloat16_rn(fmaf(cur_sc_u, zu, d));
-            }
+        if (sync_step) {
+            ok = epilogue(t, cur, cur_sc_w, cur_sc_u, false);
+        } else {
+            // the epilogue runs one step behind the MMAs
+            if (pend >= 0) ok = epilogue(pend, step_info(p, blk_lo, nblk, pend), scp_w, scp_u, true);
+            pend = t;
+            scp_w = cur_sc_w;
+            scp_u = cur_sc_u;
         }
-        buf ^= 1;
+        if (!ok) break;
     }
+    if (ok && pend >= 0) ok = epilogue(pend, step_info(p, blk_lo, nblk, pend), scp_w, scp_u, true);
 
     // Copies still in flight (only after an abort) land before the CTA exits.
     while (consumed < issued) {
@@ -1140,7 +1248,9 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
         }
         v_bytes = bytes > v_bytes ? bytes : v_bytes;
     }
-    p.a.lag = p.a.t_mode == kTGrid ? (min_blocks < kDecodeMaxLag ? (min_blocks < 1 ? 1 : min_blocks) : kDecodeMaxLag) : 0;
+    // grid mode: partial sums in step 1, the reduction in step 2, T loaded in
+    // step 3, where the U part of block 0 runs
+    p.a.lag = p.a.t_mode == kTGrid ? kDecodeMaxLag : 0;
     p.a.x_ld = p.a.K + 8;
 
     // Shared memory: the compact variant (two CTAs per SM) for calls whose
@@ -1157,28 +1267,52 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
         p.a.x_smem = 1;
         p.a.v_stage = 0;
         p.a.v_bytes = 0;
+        p.a.v_in_ring = 0;
         if (smem_layout(p.a, NT).total > budget) {
             if (small) continue;
             p.a.x_smem = 0;
         }
+        // Most ring slots that fit the budget with the current choices.
+        auto grow_slots = [&]() {
+            p.a.slots = 1;
+            while (p.a.slots < kDecodeMaxSlots) {
+                ++p.a.slots;
+                const SmemLayout Lg = smem_layout(p.a, NT);
+                if (Lg.total > budget || Lg.ring_bytes > kMaxRingBytes) {
+                    --p.a.slots;
+                    break;
+                }
+            }
+        };
         if (v_ok && v_bytes > 0) {
-            // the staged rows plus room for the rows past the last one that a
-            // 16-row k-step reads (and masks)
+            // the staged rows plus, for a ragged K, room for the rows past the
+            // last one that a 16-row k-step reads (and masks)
+            const size_t vb = v_bytes + (p.a.K % 16 ? 16 * (size_t)max_r * 2 : 0);
             p.a.v_stage = 1;
-            p.a.v_bytes = (int)(v_bytes + 16 * (size_t)max_r * 2);
-            if (smem_layout(p.a, NT).total > budget) {
-                p.a.v_stage = 0;
-                p.a.v_bytes = 0;
+            p.a.v_bytes = (int)vb;
+            p.a.v_in_ring = 0;
+            int own_slots = 0;
+            if (smem_layout(p.a, NT).total <= budget) {
+                grow_slots();
+                own_slots = p.a.slots;
+            }
+            // or in the ring's last slot level, when that holds them and
+            // leaves more slots for the stream
+            p.a.v_in_ring = 1;
+            grow_slots();
+            const uint32_t level = (uint32_t)NW * p.a.slot_chunks * kDecodeChunkBytes;
+            const bool ring_ok = p.a.slots >= 2 && vb <= level && smem_layout(p.a, NT).total <= budget;
+            if (!(ring_ok && p.a.slots > own_slots)) {
+                p.a.v_in_ring = 0;
+                if (own_slots > 0) {
+                    p.a.slots = own_slots;
+                } else {
+                    p.a.v_stage = 0;
+                    p.a.v_bytes = 0;
+                }
             }
         }
-        while (p.a.slots < kDecodeMaxSlots) {
-            ++p.a.slots;
-            const SmemLayout Lg = smem_layout(p.a, NT);
-            if (Lg.total > budget || Lg.ring_bytes > kMaxRingBytes) {
-                --p.a.slots;
-                break;
-            }
-        }
+        if (!p.a.v_stage) grow_slots();
         if (smem_layout(p.a, NT).total > budget) return WL_ERR_UNSUPPORTED;
         plan->small = small ? 1 : 0;
         done = true;

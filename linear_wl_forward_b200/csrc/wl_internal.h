@@ -23,7 +23,7 @@ constexpr int kDecodeChunkBytes = kDecodeBlockRows * kDecodeChunkK * 2;  // 2 KB
 constexpr int kDecodeMaxSlotChunks = 4;   // a ring slot holds up to 16 rows x 256 columns
 constexpr int kDecodeMaxSlots = 4;        // ring slots per warp
 constexpr int kDecodeTMaxFloats = 12288;  // M (rounded up to 8) * (sum of ranks) in shared memory
-constexpr int kDecodeMaxLag = 2;          // blocks by which the U part of a block may trail its W0 part
+constexpr int kDecodeMaxLag = 3;          // grid T mode: blocks by which the U part of a block trails its W0 part
 
 // How a CTA obtains T = V^T x.
 enum DecodeTMode : int {
@@ -66,7 +66,8 @@ struct DecodeArgs {
     int x_smem;       // x is staged in shared memory (rows padded to x_ld elements)
     int x_ld;
     int v_stage;      // each CTA bulk-copies the V rows it needs for T into shared memory
-    int v_bytes;      // shared memory reserved for them (largest over the CTAs)
+    int v_bytes;      // shared memory they need (largest over the CTAs)
+    int v_in_ring;    // they sit in the ring's last slot level until T's sums are formed
     const __nv_bfloat16 *x;
     float *Tpart;     // kTGrid: [grid][M][t_ld] partial sums, then [M][t_ld] final T
     unsigned int *sync;  // kTGrid: [0], [1] arrival counts, [2] departures; self-resetting
