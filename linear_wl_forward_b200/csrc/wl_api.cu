@@ -234,13 +234,20 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
         if ((st = scratch(pool, kSlotT, (size_t)M * t_cols * 2, &t)) != WL_OK) return st;
         __nv_bfloat16 *Vt = static_cast<__nv_bfloat16 *>(vt);
         T = static_cast<__nv_bfloat16 *>(t);
+        TransposeVArgs ta;
+        std::memset(&ta, 0, sizeof ta);
+        ta.K = K;
+        ta.Vt = Vt;
         for (int i = 0; i < P; ++i) {
             const wl_proj &q = projs[i];
             if (q.N == 0 || q.r == 0) continue;
-            cudaError_t e = launch_transpose_v(reinterpret_cast<const __nv_bfloat16 *>(q.V), K, q.r,
-                                               round_up(q.r, 64), Vt + (size_t)t_col[i] * K, stream);
-            if (e != cudaSuccess) return WL_ERR_CUDA;
+            ta.V[ta.n] = reinterpret_cast<const __nv_bfloat16 *>(q.V);
+            ta.r[ta.n] = q.r;
+            ta.r_pad[ta.n] = round_up(q.r, 64);
+            ta.row[ta.n] = t_col[i];
+            ++ta.n;
         }
+        if (launch_transpose_v(ta, stream) != cudaSuccess) return WL_ERR_CUDA;
         // T = x V for all projections at once (plain GEMM against the stacked V^T).
         GemmParams tp;
         std::memset(&tp, 0, sizeof tp);
@@ -261,6 +268,7 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
         tp.seg[0].lr_blocks = 0;
         tp.seg[0].tile_begin = 0;
         tp.num_tiles = tp.num_m_tiles * ((t_cols + bn - 1) / bn);
+        set_gemm_stages(tp);
         tp.status = pool.words;
         tp.timeout_ns = kWaitLimitNs;
         if (launch_gemm(tp, pool.num_sms, stream) != cudaSuccess) return WL_ERR_CUDA;
@@ -268,7 +276,17 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
 
     GemmParams gp;
     std::memset(&gp, 0, sizeof gp);
-    const int bn = kGemmMaxBN;
+    // Tile width: the widest of 256, 128, 64 that still gives every SM a tile
+    // (a few-token call has one 128-row tile of x, so its work is all in N).
+    // Narrower than 64 would make the x tile, re-read per tile, outweigh W0.
+    const int m_tiles = (M + kGemmBM - 1) / kGemmBM;
+    int bn = kGemmMaxBN;
+    while (bn > 64) {
+        int n_tiles = 0;
+        for (int i = 0; i < P; ++i) n_tiles += (projs[i].N + bn - 1) / bn;
+        if (m_tiles * n_tiles >= pool.num_sms) break;
+        bn /= 2;
+    }
     if ((st = make_map(&gp.tm_a, x, K, M, K, kGemmBM)) != WL_OK) return st;
     if (t_cols > 0) {
         if ((st = make_map(&gp.tm_t, T, t_cols, M, t_cols, kGemmBM)) != WL_OK) return st;
@@ -315,6 +333,7 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
     if (tiles == 0) return WL_OK;
     gp.nseg = nseg;
     gp.num_tiles = tiles;
+    set_gemm_stages(gp);
     gp.status = pool.words;
     gp.timeout_ns = kWaitLimitNs;
     return from_cuda(launch_gemm(gp, pool.num_sms, stream));

@@ -31,9 +31,26 @@ namespace wl {
 
 namespace {
 
+// Launch with programmatic dependent launch: the kernel may start while the
+// previous kernel in the stream finishes; each kernel here waits for it
+// (griddepcontrol.wait) before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr uint32_t kABytes = kGemmBM * kGemmBK * 2;     // 16 KB
-constexpr uint32_t kBBytesMax = kGemmMaxBN * kGemmBK * 2;  // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytesMax;  // 48 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccBCol = 256;
 
@@ -64,12 +81,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const 
 }  // namespace
 
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+    // The next kernel may launch now; it waits for this grid before touching
+    // memory.  This grid's own global accesses start after the wait below.
+    pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     uint8_t *base = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-    uint64_t *full = reinterpret_cast<uint64_t *>(base + kGemmStages * kStageBytes);
-    uint64_t *empty = full + kGemmStages;
-    uint64_t *tmem_full = empty + kGemmStages;
+    const uint32_t stages = (uint32_t)p.stages, stage_bytes = (uint32_t)p.stage_bytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + stages * stage_bytes);
+    uint64_t *empty = full + stages;
+    uint64_t *tmem_full = empty + stages;
     uint64_t *tmem_empty = tmem_full + 1;
     uint64_t *drain = tmem_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -80,7 +101,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const uint32_t b_bytes = (uint32_t)p.BN * kGemmBK * 2;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGemmStages; ++i) {
+        for (uint32_t i = 0; i < stages; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
@@ -106,23 +127,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait_primary();  // the previous kernel is done: x, T and the scratch are ours
 
     if (warp == 0) {
         // ------------------------------------------------------ producer ----
-        uint32_t it = 0;
+        uint32_t it = 0, slot = 0, ph = 0;  // ring position, tracked without divisions
         bool ok = true;
         for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
             const TileInfo ti = tile_info(p, t);
             const GemmSeg &sg = p.seg[ti.seg];
             const int total = nkb + sg.lr_blocks;
             for (int kb = 0; kb < total; ++kb) {
-                const uint32_t slot = it % kGemmStages, ph = (it / kGemmStages) & 1u;
                 if (!warp_wait(&empty[slot], ph ^ 1u, p, abort_flag)) {
                     ok = false;
                     break;
                 }
                 if (lane == 0) {
-                    uint8_t *sa = base + slot * kStageBytes;
+                    uint8_t *sa = base + slot * stage_bytes;
                     uint8_t *sb = sa + kABytes;
                     mbar_arrive_expect_tx(&full[slot], kABytes + b_bytes);
                     if (kb < nkb) {
@@ -136,18 +157,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 }
                 __syncwarp();
                 ++it;
+                if (++slot == stages) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
             }
         }
         if (!ok) {
             // Let the loads already issued land before the CTA exits.
-            const uint32_t inflight = it < (uint32_t)kGemmStages ? it : (uint32_t)kGemmStages;
+            const uint32_t inflight = it < stages ? it : stages;
             for (uint32_t i = it - inflight; i < it; ++i)
-                mbar_wait(&full[i % kGemmStages], (i / kGemmStages) & 1u, p.status, 1000000ull);
+                mbar_wait(&full[i % stages], (i / stages) & 1u, p.status, 1000000ull);
         }
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer ---
         const uint32_t idesc = idesc_bf16_f32(kGemmBM, p.BN);
-        uint32_t it = 0, tcount = 0;
+        uint32_t slot = 0, ph = 0, tcount = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
             const TileInfo ti = tile_info(p, t);
@@ -159,14 +184,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             }
             tc_fence_after();
             for (int kb = 0; kb < total; ++kb) {
-                const uint32_t slot = it % kGemmStages, ph = (it / kGemmStages) & 1u;
                 if (!warp_wait(&full[slot], ph, p, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t a_addr = smem_addr(base + slot * kStageBytes);
+                    const uint32_t a_addr = smem_addr(base + slot * stage_bytes);
                     const uint32_t b_addr = a_addr + kABytes;
                     const uint64_t adesc = sw128_kmajor_desc(a_addr);
                     const uint64_t bdesc = sw128_kmajor_desc(b_addr);
@@ -182,7 +206,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     tc_commit(&empty[slot]);
                 }
                 __syncwarp();
-                ++it;
+                if (++slot == stages) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
             }
             if (!ok) break;
             if (lane == 0) tc_commit(tmem_full);
@@ -258,10 +285,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
 }
 
-size_t gemm_smem_bytes() { return 1024 + kGemmStages * kStageBytes + 256; }
+// Pipeline depth for the tile width: stages of a 128 x 64 x-tile and a
+// BN x 64 W0 tile, as many as fit in 192 KB (at most kGemmMaxStages).
+void set_gemm_stages(GemmParams &p) {
+    p.stage_bytes = (int)(kABytes + (uint32_t)p.BN * kGemmBK * 2);
+    int n = (192 * 1024) / p.stage_bytes;
+    p.stages = n > kGemmMaxStages ? kGemmMaxStages : (n < 2 ? 2 : n);
+}
+
+size_t gemm_smem_bytes(const GemmParams &p) {
+    return 1024 + (size_t)p.stages * p.stage_bytes + (2 * kGemmMaxStages + 3) * 8 + 16;
+}
 
 cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
-    const size_t smem = gemm_smem_bytes();
+    const size_t smem = gemm_smem_bytes(p);
+    if (p.stages < 2 || p.stages > kGemmMaxStages || smem > 227 * 1024) return cudaErrorInvalidValue;
     // Opt in to the large shared-memory carve-out once per device.
     static bool attr_done[64] = {};
     int dev = 0;
@@ -269,21 +307,27 @@ cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
     int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
     if (grid < 1) return cudaSuccess;
-    gemm_kernel<<<grid, kGemmThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(gemm_kernel, dim3(grid), dim3(kGemmThreads), smem, stream, p);
 }
 
 // ---------------------------------------------------------- small helpers ---
-__global__ void transpose_v_kernel(const __nv_bfloat16 *__restrict__ V, int K, int r, int r_pad,
-                                   __nv_bfloat16 *__restrict__ Vt) {
+// Vt rows of every projection of a call (blockIdx.z = projection).
+__global__ void transpose_v_kernel(const __grid_constant__ TransposeVArgs a) {
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    const int pi = blockIdx.z;
+    const __nv_bfloat16 *__restrict__ V = a.V[pi];
+    const int K = a.K, r = a.r[pi], r_pad = a.r_pad[pi];
+    __nv_bfloat16 *__restrict__ Vt = a.Vt + (size_t)a.row[pi] * K;
     __shared__ __nv_bfloat16 tile[32][33];
     const int k0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
+    if (j0 >= r_pad) return;
     const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
     for (int i = ty; i < 32; i += 8) {
         const int k = k0 + i, j = j0 + tx;
@@ -296,15 +340,18 @@ __global__ void transpose_v_kernel(const __nv_bfloat16 *__restrict__ V, int K, i
     }
 }
 
-cudaError_t launch_transpose_v(const __nv_bfloat16 *V, int K, int r, int r_pad, __nv_bfloat16 *Vt,
-                               cudaStream_t stream) {
-    dim3 grid((K + 31) / 32, (r_pad + 31) / 32);
-    transpose_v_kernel<<<grid, dim3(32, 8), 0, stream>>>(V, K, r, r_pad, Vt);
-    return cudaGetLastError();
+cudaError_t launch_transpose_v(const TransposeVArgs &a, cudaStream_t stream) {
+    if (a.n < 1 || a.n > kMaxSeg) return cudaErrorInvalidValue;
+    int max_rpad = 0;
+    for (int i = 0; i < a.n; ++i) max_rpad = a.r_pad[i] > max_rpad ? a.r_pad[i] : max_rpad;
+    dim3 grid((a.K + 31) / 32, (max_rpad + 31) / 32, a.n);
+    return launch_pdl(transpose_v_kernel, grid, dim3(32, 8), 0, stream, a);
 }
 
 __global__ void pad_u_kernel(const __nv_bfloat16 *__restrict__ U, int N, int r, int r_pad,
                              __nv_bfloat16 *__restrict__ Upad) {
+    pdl_launch_dependents();
+    pdl_wait_primary();
     const size_t total = (size_t)N * r_pad;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
          i += (size_t)gridDim.x * blockDim.x) {
@@ -320,8 +367,7 @@ cudaError_t launch_pad_u(const __nv_bfloat16 *U, int N, int r, int r_pad, __nv_b
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4096) blocks = 4096;
     if (blocks < 1) return cudaSuccess;
-    pad_u_kernel<<<blocks, 256, 0, stream>>>(U, N, r, r_pad, Upad);
-    return cudaGetLastError();
+    return launch_pdl(pad_u_kernel, dim3(blocks), dim3(256), 0, stream, U, N, r, r_pad, Upad);
 }
 
 }  // namespace wl

@@ -108,7 +108,7 @@ wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;         // 128 bytes of bf16: one swizzle row
 constexpr int kGemmMaxBN = 256;
-constexpr int kGemmStages = 4;
+constexpr int kGemmMaxStages = 8;
 constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 
 struct GemmSeg {
@@ -130,19 +130,30 @@ struct GemmParams {
     int nseg;
     int M, K;
     int BN;
+    int stages;       // pipeline depth (set_gemm_stages)
+    int stage_bytes;
     int num_m_tiles;
     int num_tiles;
     int *status;
     unsigned long long timeout_ns;
 };
 
-size_t gemm_smem_bytes();
+void set_gemm_stages(GemmParams &p);
+size_t gemm_smem_bytes(const GemmParams &p);
 cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream);
 
-// Vt[j][k] = V[k][j] for j < r, 0 for r <= j < r_pad (rows of the stacked
-// transposed V, one projection per call).
-cudaError_t launch_transpose_v(const __nv_bfloat16 *V, int K, int r, int r_pad,
-                               __nv_bfloat16 *Vt, cudaStream_t stream);
+// Vt[row_p + j][k] = V_p[k][j] for j < r_p, 0 for r_p <= j < r_pad_p: the
+// stacked transposed V of every projection of a call, in one launch.
+struct TransposeVArgs {
+    const __nv_bfloat16 *V[kMaxSeg];
+    int r[kMaxSeg];
+    int r_pad[kMaxSeg];
+    int row[kMaxSeg];  // first row of projection p in Vt
+    int n;
+    int K;
+    __nv_bfloat16 *Vt;
+};
+cudaError_t launch_transpose_v(const TransposeVArgs &a, cudaStream_t stream);
 // Copy U (N x r) into Upad (N x r_pad) with zero columns beyond r.
 cudaError_t launch_pad_u(const __nv_bfloat16 *U, int N, int r, int r_pad,
                          __nv_bfloat16 *Upad, cudaStream_t stream);
