@@ -207,6 +207,29 @@ __host__ __device__ __forceinline__ void warp_u_chunks(int r, int w, int &lo, in
     warp_chunks((r + CK - 1) / CK, NW - 1 - w, lo, hi);
 }
 
+// Blocks [b0, b1) of projection sp among blocks [blk_lo, blk_hi) (empty if none).
+__host__ __device__ __forceinline__ void seg_block_range(const DecodeSeg &sg, int blk_lo, int blk_hi, int &b0,
+                                                         int &b1) {
+    const int nb = (sg.N + kDecodeBlockRows - 1) / kDecodeBlockRows;
+    b0 = sg.blk_begin > blk_lo ? sg.blk_begin : blk_lo;
+    b1 = sg.blk_begin + nb < blk_hi ? sg.blk_begin + nb : blk_hi;
+    if (b1 < b0) b1 = b0;
+}
+
+// Staged U (u_stage): the U rows of the CTA's blocks, projection after
+// projection, each block a full 16 rows (rows past N are never copied).
+// Byte offset of projection sp's rows in that region.
+__host__ __device__ inline uint32_t u_stage_off(const DecodeArgs &p, int sp, int blk_lo, int blk_hi) {
+    uint32_t off = 0;
+    for (int i = 0; i < sp; ++i) {
+        if (p.seg[i].r == 0) continue;
+        int b0, b1;
+        seg_block_range(p.seg[i], blk_lo, blk_hi, b0, b1);
+        off += (uint32_t)(b1 - b0) * kDecodeBlockRows * (uint32_t)p.seg[i].r * 2u;
+    }
+    return off;
+}
+
 // A warp's position in its sequence of ring copies.  The CTA's work is a list
 // of steps t = 0 .. nblk + lag - 1; step t holds the W0 part of the CTA's
 // block t (t < nblk) and then the U part of its block t - lag (t >= lag, when
@@ -237,7 +260,7 @@ __device__ __forceinline__ void seq_load(const DecodeArgs &p, int w, int w0_slot
         return;
     }
     const int r = p.seg[B.sp].r;
-    if (!p.u_bulk || r == 0) return;
+    if (!p.u_bulk || p.u_stage || r == 0) return;
     warp_u_chunks(r, w, q.u_lo, q.u_hi);
     q.ns = (q.u_hi - q.u_lo + p.slot_chunks - 1) / p.slot_chunks;
 }
@@ -351,6 +374,36 @@ __device__ __forceinline__ void u_chunk(float (&acu)[NT][4], uint32_t cbase, con
         ldmatrix_x4(cbase + swz[kq], a);
         const int j = kk + 2 * q;
         const bool hi_ok = kk + 8 < r;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
+            if (nvalid[nt]) {
+                const float *tr = T + (size_t)(nt * 8 + g) * t_ld;
+                t0 = tr[j];
+                t1 = tr[j + 1];
+                if (hi_ok) {
+                    t2 = tr[j + 8];
+                    t3 = tr[j + 9];
+                }
+            }
+            mma_split_t(acu[nt], a, t0, t1, t2, t3);
+        }
+    }
+}
+
+// U T for columns [j0, j1) of the rank r (16 at a time) with A = the block's
+// 16 staged U rows (row-major, row stride r) read by ldmatrix; urow_lane is
+// this lane's row (lane & 15) and column half (lane >> 4) address.  Columns
+// past r in a 16-column step are cleared (they would read the next row).
+template <int NT>
+__device__ __forceinline__ void u_staged(float (&acu)[NT][4], uint32_t urow_lane, int j0, int j1, int r,
+                                         const float *T, int t_ld, int g, int q, const bool (&nvalid)[NT]) {
+    for (int kk = j0; kk < j1; kk += 16) {
+        uint32_t a[4];
+        ldmatrix_x4(urow_lane + (uint32_t)kk * 2u, a);
+        const bool hi_ok = kk + 8 < r;
+        if (!hi_ok) a[2] = a[3] = 0u;
+        const int j = kk + 2 * q;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
@@ -658,7 +711,7 @@ __device__ bool grid_t_load(const DecodeArgs &p, int blk_lo, int blk_hi, float *
 constexpr uint32_t kArgsBytes = (uint32_t)((sizeof(DecodeArgs) + 15) & ~size_t(15));
 
 struct SmemLayout {
-    uint32_t slot_bytes, ring_bytes, ts_off, red_off, xs_off, vs_off, zs_off, bar_off, flag_off, total;
+    uint32_t slot_bytes, ring_bytes, ts_off, red_off, xs_off, vs_off, us_off, zs_off, bar_off, flag_off, total;
 };
 
 // Shared memory opens with the copy of the arguments; the ring starts at the
@@ -678,9 +731,12 @@ __host__ __device__ inline SmemLayout smem_layout(const DecodeArgs &p, int NT) {
     L.vs_off = L.xs_off + ((x_bytes + 127u) & ~127u);
     const uint32_t v_bytes = (p.v_stage && !p.v_in_ring) ? (uint32_t)p.v_bytes : 0u;
     L.zs_off = L.vs_off + ((v_bytes + 127u) & ~127u);
+    const uint32_t u_bytes = p.u_stage ? (uint32_t)p.u_bytes : 0u;
+    L.us_off = L.zs_off;
+    L.zs_off = L.us_off + ((u_bytes + 127u) & ~127u);
     const uint32_t z_bytes = p.lag > 0 ? (uint32_t)(p.lag + 1) * BR * p.M * 4u : 0u;
     L.bar_off = L.zs_off + ((z_bytes + 127u) & ~127u);
-    L.flag_off = L.bar_off + (uint32_t)(NW * p.slots + 5) * 8u;
+    L.flag_off = L.bar_off + (uint32_t)(NW * p.slots + 6) * 8u;
     L.total = L.flag_off + 16u + 1024u + kArgsBytes;  // + the copy of the arguments, before the ring
     return L;
 }
@@ -773,6 +829,8 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     uint64_t *vbar = full + NW * SLOTS;  // V rows staged
     uint64_t *red_full = vbar + 1;       // [2] every warp's sums of a step are in
     uint64_t *red_empty = vbar + 3;      // [2] the step's epilogue has read them
+    uint64_t *ubar = vbar + 5;           // U rows staged
+    const uint8_t *us = smem + L.us_off;  // staged U rows (u_stage)
     // staged V rows: their own region, or the ring's last slot level (handed
     // to the W0 stream once T's sums are formed)
     uint8_t *vs = p.v_in_ring ? smem + (size_t)(SLOTS - 1) * NW * L.slot_bytes : smem + L.vs_off;
@@ -784,6 +842,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
 
     if (tid == 0) {
         for (int i = 0; i < NW * SLOTS + 1; ++i) mbar_init(&full[i], 1);
+        mbar_init(ubar, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&red_full[i], NW);
             mbar_init(&red_empty[i], (BR * p.M + 31) / 32);
@@ -838,6 +897,30 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             const uint32_t bytes = (uint32_t)(k1 - k0) * (uint32_t)p.seg[sp].r * 2u;
             if (bytes) bulk_load(vs + off, p.seg[sp].V + (size_t)k0 * p.seg[sp].r, bytes, vbar);
             off += bytes;
+        }
+    }
+    if (p.u_stage && tid == 32) {
+        // the U rows of this CTA's blocks (full 16-row blocks in shared memory;
+        // only rows below N are copied)
+        uint32_t total = 0;
+        for (int sp = 0; sp < p.nseg; ++sp) {
+            const DecodeSeg &sg = p.seg[sp];
+            if (sg.r == 0) continue;
+            int b0, b1;
+            seg_block_range(sg, blk_lo, blk_hi, b0, b1);
+            const int r0 = (b0 - sg.blk_begin) * BR, r1 = min(sg.N, (b1 - sg.blk_begin) * BR);
+            if (r1 > r0) total += (uint32_t)(r1 - r0) * (uint32_t)sg.r * 2u;
+        }
+        mbar_arrive_expect_tx(ubar, total);
+        for (int sp = 0; sp < p.nseg; ++sp) {
+            const DecodeSeg &sg = p.seg[sp];
+            if (sg.r == 0) continue;
+            int b0, b1;
+            seg_block_range(sg, blk_lo, blk_hi, b0, b1);
+            const int r0 = (b0 - sg.blk_begin) * BR, r1 = min(sg.N, (b1 - sg.blk_begin) * BR);
+            if (r1 > r0)
+                bulk_load(const_cast<uint8_t *>(us) + u_stage_off(p, sp, blk_lo, blk_hi),
+                          sg.U + (size_t)r0 * sg.r, (uint32_t)(r1 - r0) * (uint32_t)sg.r * 2u, ubar);
         }
     }
     // the whole ring, less the level that holds V until T's sums are formed
@@ -895,6 +978,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
         xg_lane[nt] = p.x + (size_t)nn * K + 2 * q;
     }
 
+    bool u_ready = false;  // the staged U rows have been waited for
     uint32_t consumed = 0;
     int csl = 0;       // ring slot of the next copy to consume
     uint32_t cph = 0;  // its barrier phase parity
@@ -1009,7 +1093,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
         // ---- U part of block t - lag: U T ----
         const bool u_part = S.has_u && S.ru > 0;
         const DecodeSeg &sgu = p.seg[S.bu.sp];
-        if (u_part && p.u_bulk && ok) {
+        if (u_part && p.u_bulk && !p.u_stage && ok) {
             int u_lo, u_hi;
             warp_u_chunks(S.ru, warp, u_lo, u_hi);
             const int nu = (u_hi - u_lo + SC - 1) / SC;
@@ -1025,6 +1109,24 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
                     u_chunk<NT>(acu, sbase + (uint32_t)cc * kDecodeChunkBytes, swz, (c_lo + cc) * CK, S.ru,
                                 Ts + sgu.t_off, p.t_ld, g, q, nvalid);
                 release_slot();
+            }
+        }
+        if (u_part && p.u_stage && ok) {
+            if (!u_ready) {
+                ok = warp_wait(ubar, 0, p, abort_flag);
+                u_ready = true;
+            }
+            if (ok) {
+                int u_lo, u_hi;
+                warp_u_chunks(S.ru, warp, u_lo, u_hi);
+                int b0, b1;
+                seg_block_range(sgu, blk_lo, blk_hi, b0, b1);
+                // this lane's ldmatrix row (lane & 15) and column half of the block
+                const uint32_t urow = smem_addr(us) + u_stage_off(p, S.bu.sp, blk_lo, blk_hi) +
+                                      (uint32_t)(((S.bu.row0 - (b0 - sgu.blk_begin) * BR) + (lane & 15)) * S.ru +
+                                                 (lane >> 4) * 8) * 2u;
+                u_staged<NT>(acu, urow, u_lo * CK, min(S.ru, u_hi * CK), S.ru, Ts + sgu.t_off, p.t_ld, g, q,
+                             nvalid);
             }
         }
         if (u_part && !p.u_bulk && ok) {
@@ -1125,6 +1227,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
         }
     }
     if (tid == 0 && p.v_stage) mbar_wait(vbar, 0, p.status, 1000000ull);
+    if (tid == 32 && p.u_stage) mbar_wait(ubar, 0, p.status, 1000000ull);
 }
 
 // ------------------------------------------------------------------ host ---
@@ -1234,7 +1337,7 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
         }
     }
     int min_blocks = blocks, max_blocks = 0;
-    size_t v_bytes = 0;
+    size_t v_bytes = 0, u_bytes = 0;
     for (int c = 0; c < grid; ++c) {
         int lo, hi;
         cta_blocks(p.a, c, grid, lo, hi);
@@ -1247,6 +1350,14 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
             bytes += (size_t)(k1 - k0) * p.a.seg[i].r * 2;
         }
         v_bytes = bytes > v_bytes ? bytes : v_bytes;
+        size_t ub = 0;
+        for (int i = 0; i < p.a.nseg; ++i) {
+            if (p.a.seg[i].r == 0) continue;
+            int b0, b1;
+            seg_block_range(p.a.seg[i], lo, hi, b0, b1);
+            ub += (size_t)(b1 - b0) * BR * p.a.seg[i].r * 2;
+        }
+        u_bytes = ub > u_bytes ? ub : u_bytes;
     }
     // grid mode: partial sums in step 1, the reduction in step 2, T loaded in
     // step 3, where the U part of block 0 runs
@@ -1268,6 +1379,8 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
         p.a.v_stage = 0;
         p.a.v_bytes = 0;
         p.a.v_in_ring = 0;
+        p.a.u_stage = 0;
+        p.a.u_bytes = 0;
         if (smem_layout(p.a, NT).total > budget) {
             if (small) continue;
             p.a.x_smem = 0;
@@ -1313,6 +1426,20 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
             }
         }
         if (!p.a.v_stage) grow_slots();
+        if (small && p.a.u_bulk && u_bytes > 0 && !p.a.v_in_ring) {
+            // the compact variant's ring is shallow: U rides outside it
+            const int slots = p.a.slots;
+            p.a.u_stage = 1;
+            p.a.u_bytes = (int)u_bytes;
+            p.a.slots = 1;
+            if (smem_layout(p.a, NT).total > budget) {
+                p.a.u_stage = 0;
+                p.a.u_bytes = 0;
+                p.a.slots = slots;
+            } else {
+                grow_slots();
+            }
+        }
         if (smem_layout(p.a, NT).total > budget) return WL_ERR_UNSUPPORTED;
         plan->small = small ? 1 : 0;
         done = true;

@@ -68,6 +68,8 @@ struct DecodeArgs {
     int v_stage;      // each CTA bulk-copies the V rows it needs for T into shared memory
     int v_bytes;      // shared memory they need (largest over the CTAs)
     int v_in_ring;    // they sit in the ring's last slot level until T's sums are formed
+    int u_stage;      // each CTA bulk-copies its blocks' U rows into shared memory (not through the ring)
+    int u_bytes;      // shared memory they need (largest over the CTAs)
     const __nv_bfloat16 *x;
     float *Tpart;     // kTGrid: [grid][M][t_ld] partial sums, then [M][t_ld] final T
     unsigned int *sync;  // kTGrid: [0], [1] arrival counts, [2] departures; self-resetting
