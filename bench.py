@@ -120,15 +120,21 @@ def launches_per_call(call, path):
         return 1  # one fused kernel: W0 x, V^T x and the epilogue
     n = 1
     if any(rs):
-        n += sum(1 for r in rs if r) + 1  # V transposes + the T = x V GEMM
+        n += 2  # one V transpose for all projections + the T = x V GEMM
         n += sum(1 for r in rs if r and r % 8)  # padded U copies
     return n
 
 
 def call_path(call):
+    """The kernel path the library's automatic choice takes for a call (the
+    rule of wl_path in include/wl.h)."""
     import linear_wl_forward_b200 as wl
 
-    return "decode" if call.x.shape[0] <= wl.DECODE_MAX_M else "gemm"
+    M = call.x.shape[0]
+    rows = sum(p.N for p in call.projs)
+    if M <= 4 or (M <= wl.DECODE_MAX_M and rows < 8192):
+        return "decode"
+    return "gemm"
 
 
 # ------------------------------------------------------------- workloads --

@@ -75,8 +75,10 @@ typedef struct {
     int r;             /* rank of the delta, 0 <= r <= WL_MAX_RANK     */
 } wl_proj;
 
-/* Which kernels a forward call uses.  WL_PATH_AUTO picks by M; the others exist
- * so tests and benchmarks can exercise each kernel on any shape. */
+/* Which kernels a forward call uses.  WL_PATH_AUTO takes the decode kernel for
+ * M <= 4, and for M <= WL_DECODE_MAX_M when the call's projections total fewer
+ * than 8192 output rows; otherwise the tensor-core GEMM.  The others exist so
+ * tests and benchmarks can exercise each kernel on any shape. */
 typedef enum {
     WL_PATH_AUTO = 0,
     WL_PATH_DECODE = 1, /* weight-streaming kernel (bulk copies + warp MMA), 1 <= M <= WL_DECODE_MAX_M */

@@ -167,6 +167,23 @@ wl_status validate(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, 
 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
+// WL_PATH_AUTO: the weight-streaming decode kernel for up to 4 tokens, and
+// for up to WL_DECODE_MAX_M tokens when the call is narrow (its projections
+// total fewer than 8192 output rows).  Wider calls with 5..16 tokens go to the
+// tensor-core GEMM, which keeps x out of shared memory and fills every SM with
+// tiles; measured on B200 (one call at a time, rotating buffers > L2):
+//   stacked gate/up 2 x 21504 x 5376, M = 8 / 16: GEMM 162 / 152 us, decode 252 / 242 us
+//   stacked gate/up 2 x 4096 x 1152, M = 8: GEMM 26.9 us, decode 30.1 us
+//   down 5376 x 21504, M = 8 / 16: decode 107 / 141 us, GEMM 231 / 234 us
+//   q/k/v 1536 x 1152, M = 8: decode 19.5 us, GEMM 22.9 us
+bool auto_decode(int M, const wl_proj *projs, int P) {
+    if (M > WL_DECODE_MAX_M) return false;
+    if (M <= 4) return true;
+    long long rows = 0;
+    for (int i = 0; i < P; ++i) rows += projs[i].N;
+    return rows < 8192;
+}
+
 // ------------------------------------------------------------------ paths --
 // Fills the decode parameters of a call; false if no projection has rows.
 bool build_decode_params(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
@@ -357,7 +374,7 @@ wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, w
     std::lock_guard<std::mutex> lock(g_mu);
     DevicePool *pool = nullptr;
     if ((st = pool_for_current_device(&pool)) != WL_OK) return st;
-    if (path == WL_PATH_AUTO && M <= WL_DECODE_MAX_M) {
+    if (path == WL_PATH_AUTO && auto_decode(M, projs, P)) {
         // The decode kernel declines shapes it cannot hold (before launching
         // anything); those go to the tensor-core GEMM.
         st = run_decode(*pool, x, M, K, projs, P, stream);
