@@ -290,7 +290,13 @@ def secondary_figures(wl, peaks):
         "us_per_call": round(ms * 1e3, 2), "weight_bytes_per_call": b}
     del dev, outs, g
     torch.cuda.empty_cache()
-    # Gemma-4-31B prefill, M = 4096: stacked gate/up of layer 0
+    out["gemma4_prefill_gate_up_M4096"] = prefill_figure(wl, peaks)
+    return out
+
+
+def prefill_figure(wl, peaks):
+    """Gemma-4-31B prefill, M = 4096: the stacked gate/up call of layer 0
+    (2 x 21504 x 5376, rank 256) on the tensor-core path."""
     calls = wl_inputs.gemma4_calls(seed=5, r=256, M=4096, layers=[0], families=("gate",))
     dev = [to_dev_call(c) for c in calls]
     outs, _ = alloc_outputs(calls)
@@ -299,10 +305,8 @@ def secondary_figures(wl, peaks):
     c = calls[0]
     fl = sum(footprint.call_flops(4096, p.N, p.K, p.r) for p in c.projs)
     tf = fl / (ms * 1e-3) / 1e12
-    out["gemma4_prefill_gate_up_M4096"] = {
-        "TFLOP/s": round(tf, 1), "tc_frac": round(tf / peaks["bf16_tflops"], 4),
-        "ms_per_call": round(ms, 3), "flops_per_call": fl, "peak": peaks["bf16_tflops"]}
-    return out
+    return {"TFLOP/s": round(tf, 1), "tc_frac": round(tf / peaks["bf16_tflops"], 4),
+            "ms_per_call": round(ms, 3), "flops_per_call": fl, "peak": peaks["bf16_tflops"]}
 
 
 # ---------------------------------------------------------- CPU baseline --
@@ -393,6 +397,8 @@ def main():
                     help="time only the dominant kernel's call (the command the ncu summaries profile)")
     ap.add_argument("--call", default="gemma3_gate_up", choices=sorted(ROOFLINE_CALLS),
                     help="the call --roofline-only times")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the Gemma-4-31B gate/up prefill call (the command the GEMM ncu summary profiles)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -417,6 +423,9 @@ def main():
     peaks = load_peaks()
     if args.roofline_only:
         print(json.dumps({"roofline": decode_roofline(wl, peaks, args.call)}), flush=True)
+        return
+    if args.prefill_only:
+        print(json.dumps({"prefill": prefill_figure(wl, peaks)}), flush=True)
         return
 
     calls, wbytes, flops, desc = build_workload(args.workload)
