@@ -77,7 +77,15 @@ wl_status make_map(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per device-side wait
 constexpr int kMaxDevices = 64;
 
-enum Slot { kSlotT = 0, kSlotTPart, kSlotVt, kSlotUPad0, kNumSlots = kSlotUPad0 + kMaxSeg };
+enum Slot {
+    kSlotT = 0,
+    kSlotTPart,
+    kSlotVt,
+    kSlotPart,
+    kSlotTileCnt,  // zeroed when allocated; the kernels leave it zero
+    kSlotUPad0,
+    kNumSlots = kSlotUPad0 + kMaxSeg
+};
 
 struct DevicePool {
     bool ready = false;
@@ -114,7 +122,7 @@ wl_status pool_for_current_device(DevicePool **out) {
 
 // Grow-only scratch.  Growing waits for the device so no kernel still uses
 // the old buffer; steady-state calls of one shape never reach cudaMalloc.
-wl_status scratch(DevicePool &p, int slot, size_t bytes, void **out) {
+wl_status scratch(DevicePool &p, int slot, size_t bytes, void **out, bool zeroed = false) {
     if (bytes == 0) bytes = 16;
     if (p.cap[slot] < bytes) {
         size_t want = std::max(bytes, p.cap[slot] * 2);
@@ -129,6 +137,7 @@ wl_status scratch(DevicePool &p, int slot, size_t bytes, void **out) {
             cudaGetLastError();
             return WL_ERR_NOMEM;
         }
+        if (zeroed && cudaMemset(p.buf[slot], 0, want) != cudaSuccess) return WL_ERR_CUDA;
         p.cap[slot] = want;
     }
     *out = p.buf[slot];
@@ -285,6 +294,8 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
         tp.seg[0].lr_blocks = 0;
         tp.seg[0].tile_begin = 0;
         tp.num_tiles = tp.num_m_tiles * ((t_cols + bn - 1) / bn);
+        tp.ksplit = 1;
+        tp.kb_split = (K + kGemmBK - 1) / kGemmBK;
         set_gemm_stages(tp);
         tp.status = pool.words;
         tp.timeout_ns = kWaitLimitNs;
@@ -293,27 +304,38 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
 
     GemmParams gp;
     std::memset(&gp, 0, sizeof gp);
-    // Tile width: the widest of 256, 128, 64 that still gives every SM a tile
-    // (a few-token call has one 128-row tile of x, so its work is all in N).
-    // Narrower than 64 would make the x tile, re-read per tile, outweigh W0.
-    const int m_tiles = (M + kGemmBM - 1) / kGemmBM;
+    const int nkb = (K + kGemmBK - 1) / kGemmBK;
+    const bool swap = M <= kGemmSwapMaxM;
     int bn = kGemmMaxBN;
-    while (bn > 64) {
-        int n_tiles = 0;
-        for (int i = 0; i < P; ++i) n_tiles += (projs[i].N + bn - 1) / bn;
-        if (m_tiles * n_tiles >= pool.num_sms) break;
-        bn /= 2;
+    if (swap) {
+        // Few tokens: swap the operands so the 128-row MMA side runs over the
+        // output rows (W0 / U tiles) and the tokens are the MMA's N (mp).
+        bn = kGemmBM;
+        gp.swap = 1;
+        gp.mp = round_up(M, 16);
+    } else {
+        // Tile width: the widest of 256, 128, 64 that still gives every SM a
+        // tile.  Narrower than 64 would make the x tile, re-read per tile,
+        // outweigh W0.
+        const int m_tiles = (M + kGemmBM - 1) / kGemmBM;
+        while (bn > 64) {
+            int n_tiles = 0;
+            for (int i = 0; i < P; ++i) n_tiles += (projs[i].N + bn - 1) / bn;
+            if (m_tiles * n_tiles >= pool.num_sms) break;
+            bn /= 2;
+        }
     }
-    if ((st = make_map(&gp.tm_a, x, K, M, K, kGemmBM)) != WL_OK) return st;
+    const uint32_t xb_rows = swap ? (uint32_t)gp.mp : (uint32_t)kGemmBM;
+    if ((st = make_map(&gp.tm_a, x, K, M, K, xb_rows)) != WL_OK) return st;
     if (t_cols > 0) {
-        if ((st = make_map(&gp.tm_t, T, t_cols, M, t_cols, kGemmBM)) != WL_OK) return st;
+        if ((st = make_map(&gp.tm_t, T, t_cols, M, t_cols, xb_rows)) != WL_OK) return st;
     } else {
         gp.tm_t = gp.tm_a;
     }
     gp.M = M;
     gp.K = K;
     gp.BN = bn;
-    gp.num_m_tiles = (M + kGemmBM - 1) / kGemmBM;
+    gp.num_m_tiles = swap ? 1 : (M + kGemmBM - 1) / kGemmBM;
     int tiles = 0, nseg = 0;
     for (int i = 0; i < P; ++i) {
         const wl_proj &q = projs[i];
@@ -350,6 +372,33 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
     if (tiles == 0) return WL_OK;
     gp.nseg = nseg;
     gp.num_tiles = tiles;
+    // K ranges per tile: in swap mode, enough to fill the SMs when the output
+    // rows alone give too few tiles (each range keeps >= 8 K blocks).
+    // Only when the output tiles alone leave SMs idle; the smallest split that
+    // keeps 80% of the SMs busy (the ranges' sums cost a reduction).
+    gp.ksplit = 1;
+    if (swap && tiles < pool.num_sms) {
+        for (int ks = 2; ks <= kGemmMaxKSplit; ++ks) {
+            const int kbs = (nkb + ks - 1) / ks;
+            if (kbs < 8) break;
+            const int eff_ks = (nkb + kbs - 1) / kbs;
+            const long long u = (long long)tiles * eff_ks;
+            const long long waves = (u + pool.num_sms - 1) / pool.num_sms;
+            gp.ksplit = eff_ks;
+            if ((double)u / (double)(waves * pool.num_sms) >= 0.8) break;
+        }
+    }
+    gp.kb_split = (nkb + gp.ksplit - 1) / gp.ksplit;
+    gp.ksplit = (nkb + gp.kb_split - 1) / gp.kb_split;
+    if (gp.ksplit > 1) {
+        void *part = nullptr, *cnt = nullptr;
+        const size_t pf = (size_t)(gp.ksplit + 1) * tiles * gp.mp * kGemmBM;
+        if ((st = scratch(pool, kSlotPart, pf * sizeof(float), &part)) != WL_OK) return st;
+        if ((st = scratch(pool, kSlotTileCnt, (size_t)tiles * sizeof(unsigned), &cnt, true)) != WL_OK)
+            return st;
+        gp.part = static_cast<float *>(part);
+        gp.tile_cnt = static_cast<unsigned int *>(cnt);
+    }
     set_gemm_stages(gp);
     gp.status = pool.words;
     gp.timeout_ns = kWaitLimitNs;
@@ -437,6 +486,9 @@ wl_status wl_last_device_status(void *stream) {
     // A kernel that gave up may have left its arrival counters set: clear the
     // whole word block (status and counters) after an error.
     if (word != 0 && cudaMemset(pool->words, 0, 64 * sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
+    if (word != 0 && pool->buf[wl::kSlotTileCnt] &&
+        cudaMemset(pool->buf[wl::kSlotTileCnt], 0, pool->cap[wl::kSlotTileCnt]) != cudaSuccess)
+        return WL_ERR_CUDA;
     return static_cast<wl_status>(word);
 }
 

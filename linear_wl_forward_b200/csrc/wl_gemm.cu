@@ -1,5 +1,6 @@
-// Tensor-core path (any M; chosen for M > 4): a persistent tcgen05 GEMM whose
-// epilogue applies the per-row scale and adds the rank-r term,
+// Tensor-core path (any M; see wl_path for when it is chosen): a persistent
+// tcgen05 GEMM whose epilogue applies the per-row scale and adds the rank-r
+// term,
 //
 //     y[m][n] = s[n] * sum_k x[m][k] W0[n][k]  +  sum_j T[m][j] U[n][j],
 //     T = x V (computed first by the same kernel in plain mode, bf16 output).
@@ -19,6 +20,15 @@
 //               bf16, stores with edge checks.
 // The scale touches only the shared-block product, so the two products keep
 // separate accumulators; U V^T is never formed.
+//
+// Swap-AB mode (few tokens, M <= 16): the 128-row side of the MMA runs over
+// output rows instead -- A = 128 x 64 tiles of W0 (then U), B = x (then T)
+// tiles of mp = M rounded up to 16 rows, D = 128 rows x mp tokens -- so a
+// tile streams 128 full rows of W0 and no MMA lanes are spent on absent
+// tokens.  When the output rows alone give fewer tiles than SMs, K is cut
+// into ranges (at most 8, each >= 8 blocks) whose sums are stored; the CTA
+// that completes a tile's arrival count adds them up in range order
+// (deterministic) and writes y.
 //
 // Bf16 operands with fp32 accumulation follow "Quality (Gemma 4 31B)", "Kernel
 // optimizations", GEMM path item 2 (bf16 matmuls accumulate in fp32 on the
@@ -95,10 +105,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     uint64_t *drain = tmem_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *last_flag = abort_flag + 1;  // swap mode: this CTA adds up the tile's K ranges
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = (p.K + kGemmBK - 1) / kGemmBK;
-    const uint32_t b_bytes = (uint32_t)p.BN * kGemmBK * 2;
+    // Operand B rows per stage: W0 / U tiles of BN rows, or (swap) x / T
+    // tiles of mp rows; operand A is always 128 rows (x / T, or W0 / U).
+    const uint32_t b_rows = p.swap ? (uint32_t)p.mp : (uint32_t)p.BN;
+    const uint32_t b_bytes = b_rows * kGemmBK * 2;
+    const int units = p.num_tiles * p.ksplit;
 
     if (threadIdx.x == 0) {
         for (uint32_t i = 0; i < stages; ++i) {
@@ -133,11 +148,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         // ------------------------------------------------------ producer ----
         uint32_t it = 0, slot = 0, ph = 0;  // ring position, tracked without divisions
         bool ok = true;
-        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-            const TileInfo ti = tile_info(p, t);
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const int tile = u / p.ksplit, split = u - tile * p.ksplit;
+            const TileInfo ti = tile_info(p, tile);
             const GemmSeg &sg = p.seg[ti.seg];
-            const int total = nkb + sg.lr_blocks;
-            for (int kb = 0; kb < total; ++kb) {
+            const int kb0 = split * p.kb_split;
+            const int kb1 = min(nkb, kb0 + p.kb_split);
+            const int lr = split == 0 ? sg.lr_blocks : 0;
+            const int total = (kb1 - kb0) + lr;
+            for (int i = 0; i < total; ++i) {
                 if (!warp_wait(&empty[slot], ph ^ 1u, p, abort_flag)) {
                     ok = false;
                     break;
@@ -146,13 +165,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     uint8_t *sa = base + slot * stage_bytes;
                     uint8_t *sb = sa + kABytes;
                     mbar_arrive_expect_tx(&full[slot], kABytes + b_bytes);
-                    if (kb < nkb) {
-                        tma_load_2d(sa, &p.tm_a, kb * kGemmBK, ti.m0, &full[slot]);
-                        tma_load_2d(sb, &p.tm_b[ti.seg], kb * kGemmBK, ti.n0, &full[slot]);
+                    if (i < kb1 - kb0) {
+                        const int kc = (kb0 + i) * kGemmBK;
+                        if (p.swap) {
+                            tma_load_2d(sa, &p.tm_b[ti.seg], kc, ti.n0, &full[slot]);
+                            tma_load_2d(sb, &p.tm_a, kc, 0, &full[slot]);
+                        } else {
+                            tma_load_2d(sa, &p.tm_a, kc, ti.m0, &full[slot]);
+                            tma_load_2d(sb, &p.tm_b[ti.seg], kc, ti.n0, &full[slot]);
+                        }
                     } else {
-                        const int j0 = (kb - nkb) * kGemmBK;
-                        tma_load_2d(sa, &p.tm_t, sg.t_col + j0, ti.m0, &full[slot]);
-                        tma_load_2d(sb, &p.tm_u[ti.seg], j0, ti.n0, &full[slot]);
+                        const int j0 = (i - (kb1 - kb0)) * kGemmBK;
+                        if (p.swap) {
+                            tma_load_2d(sa, &p.tm_u[ti.seg], j0, ti.n0, &full[slot]);
+                            tma_load_2d(sb, &p.tm_t, sg.t_col + j0, 0, &full[slot]);
+                        } else {
+                            tma_load_2d(sa, &p.tm_t, sg.t_col + j0, ti.m0, &full[slot]);
+                            tma_load_2d(sb, &p.tm_u[ti.seg], j0, ti.n0, &full[slot]);
+                        }
                     }
                 }
                 __syncwarp();
@@ -171,19 +201,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer ---
-        const uint32_t idesc = idesc_bf16_f32(kGemmBM, p.BN);
+        const uint32_t idesc = idesc_bf16_f32(kGemmBM, b_rows);
         uint32_t slot = 0, ph = 0, tcount = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-            const TileInfo ti = tile_info(p, t);
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const int tile = u / p.ksplit, split = u - tile * p.ksplit;
+            const TileInfo ti = tile_info(p, tile);
             const GemmSeg &sg = p.seg[ti.seg];
-            const int total = nkb + sg.lr_blocks;
+            const int kb0 = split * p.kb_split;
+            const int nmain = min(nkb, kb0 + p.kb_split) - kb0;
+            const int total = nmain + (split == 0 ? sg.lr_blocks : 0);
             if (!warp_wait(tmem_empty, (tcount & 1u) ^ 1u, p, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            for (int kb = 0; kb < total; ++kb) {
+            for (int i = 0; i < total; ++i) {
                 if (!warp_wait(&full[slot], ph, p, abort_flag)) {
                     ok = false;
                     break;
@@ -194,9 +227,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     const uint32_t b_addr = a_addr + kABytes;
                     const uint64_t adesc = sw128_kmajor_desc(a_addr);
                     const uint64_t bdesc = sw128_kmajor_desc(b_addr);
-                    const bool lowrank = kb >= nkb;
+                    const bool lowrank = i >= nmain;
                     const uint32_t d = tmem_base + (lowrank ? kAccBCol : 0u);
-                    const bool first = (kb == 0) || (kb == nkb);
+                    const bool first = (i == 0) || (i == nmain);
 #pragma unroll
                     for (int k = 0; k < kGemmBK / 16; ++k) {
                         // advance 16 elements (32 bytes) along K inside the swizzle row
@@ -222,7 +255,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             __syncwarp();
             mbar_wait(drain, 0, p.status, 1000000ull);
         }
-    } else {
+    } else if (!p.swap) {
         // ------------------------------------------------------- epilogue ---
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int row_in_tile = q * 32 + lane;
@@ -275,6 +308,109 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             if (lane == 0) mbar_arrive(tmem_empty);
             ++tcount;
         }
+    } else {
+        // ------------------------------------------------- swap epilogue ---
+        // TMEM lane = output row n0 + lane_in_tile, column = token.  With one
+        // K range per tile: y = s * A + B directly.  With several: each range
+        // stores its sums; the CTA that completes a tile's arrival count adds
+        // the ranges up in range order (deterministic) and writes y.  The four
+        // epilogue warps then meet at named barriers, so they also decide
+        // together to stop (bar.red.or) -- none may leave one alone.
+        const int q = warp & 3;
+        const int row_in_tile = q * 32 + lane;
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+        const int mp = p.mp;
+        const size_t tile_stride = (size_t)mp * kGemmBM;
+        uint32_t tcount = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            const int tile = u / p.ksplit, split = u - tile * p.ksplit;
+            const TileInfo ti = tile_info(p, tile);
+            const GemmSeg &sg = p.seg[ti.seg];
+            bool ok = warp_wait(tmem_full, tcount & 1u, p, abort_flag);
+            if (p.ksplit > 1) {
+                uint32_t any_fail;
+                asm volatile(
+                    "{\n\t.reg .pred p, q;\n\t"
+                    "setp.ne.u32 p, %1, 0;\n\t"
+                    "bar.red.or.pred q, 1, 128, p;\n\t"
+                    "selp.u32 %0, 1, 0, q;\n\t}"
+                    : "=r"(any_fail)
+                    : "r"((uint32_t)!ok)
+                    : "memory");
+                ok = any_fail == 0;
+            }
+            if (!ok) break;
+            tc_fence_after();
+            const int n = ti.n0 + row_in_tile;
+            const bool lr = sg.lr_blocks > 0;
+            const bool lr_here = lr && split == 0;
+            const float sc = (sg.s && n < sg.N) ? __ldg(sg.s + n) : 1.f;
+            float *zp = p.part + ((size_t)split * p.num_tiles + tile) * tile_stride + row_in_tile;
+            float *dp = p.part + ((size_t)p.ksplit * p.num_tiles + tile) * tile_stride + row_in_tile;
+            for (int c = 0; c < mp; c += 32) {
+                uint32_t a[32], b[32];
+                tmem_ld32(lane_addr + (uint32_t)c, a);
+                if (lr_here) tmem_ld32(lane_addr + kAccBCol + (uint32_t)c, b);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int m = c + i;
+                    if (m >= p.M) break;
+                    const float za = __uint_as_float(a[i]);
+                    const float zb = lr_here ? __uint_as_float(b[i]) : 0.f;
+                    if (p.ksplit == 1) {
+                        if (n < sg.N) sg.y[(size_t)m * sg.ldy + n] = __float2bfloat16_rn(fmaf(sc, za, zb));
+                    } else {
+                        // [split][tile][token][row] partial sums, rows contiguous
+                        zp[(size_t)m * kGemmBM] = za;
+                        if (lr_here) dp[(size_t)m * kGemmBM] = zb;
+                    }
+                }
+            }
+            // TMEM is read: the MMA warp may start the next unit.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_empty);
+            ++tcount;
+            if (p.ksplit == 1) continue;
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (warp == 2 && lane == 0)
+                *last_flag = atomicAdd(&p.tile_cnt[tile], 1u) == (unsigned)(p.ksplit - 1) ? 1 : 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (*last_flag) {
+                __threadfence();
+                if (n < sg.N) {
+                    // eight tokens at a time, every range's value loaded before
+                    // any is added (independent loads), then added in range order
+                    const float *zr = p.part + (size_t)tile * tile_stride + row_in_tile;
+                    const size_t split_stride = (size_t)p.num_tiles * tile_stride;
+                    for (int m0 = 0; m0 < p.M; m0 += 8) {
+                        float v[kGemmMaxKSplit][8], d[8];
+#pragma unroll
+                        for (int sidx = 0; sidx < kGemmMaxKSplit; ++sidx)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                v[sidx][i] = (sidx < p.ksplit && m0 + i < p.M)
+                                                 ? __ldcg(zr + sidx * split_stride + (size_t)(m0 + i) * kGemmBM)
+                                                 : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            d[i] = (lr && m0 + i < p.M) ? __ldcg(dp + (size_t)(m0 + i) * kGemmBM) : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            if (m0 + i >= p.M) break;
+                            float z = 0.f;
+#pragma unroll
+                            for (int sidx = 0; sidx < kGemmMaxKSplit; ++sidx) z += v[sidx][i];
+                            sg.y[(size_t)(m0 + i) * sg.ldy + n] = __float2bfloat16_rn(fmaf(sc, z, d[i]));
+                        }
+                    }
+                }
+                if (warp == 2 && lane == 0) p.tile_cnt[tile] = 0u;  // for the next call
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // last_flag is reused by the next unit
+        }
     }
 
     tc_fence_before();
@@ -285,11 +421,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
 }
 
-// Pipeline depth for the tile width: stages of a 128 x 64 x-tile and a
-// BN x 64 W0 tile, as many as fit in 192 KB (at most kGemmMaxStages).
+// Pipeline depth for the tile shapes: stages of a 128 x 64 A tile and a
+// BN x 64 (or, swap, mp x 64) B tile, as many as fit in 200 KB (at most
+// kGemmMaxStages).
 void set_gemm_stages(GemmParams &p) {
-    p.stage_bytes = (int)(kABytes + (uint32_t)p.BN * kGemmBK * 2);
-    int n = (192 * 1024) / p.stage_bytes;
+    const uint32_t b_rows = p.swap ? (uint32_t)p.mp : (uint32_t)p.BN;
+    p.stage_bytes = (int)(kABytes + b_rows * kGemmBK * 2);  // multiples of 1024 (rows % 8 == 0)
+    int n = (200 * 1024) / p.stage_bytes;
     p.stages = n > kGemmMaxStages ? kGemmMaxStages : (n < 2 ? 2 : n);
 }
 
@@ -311,7 +449,9 @@ cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    if (p.ksplit < 1 || (p.swap && (p.mp < 16 || p.mp > 64 || p.mp % 16 != 0))) return cudaErrorInvalidValue;
+    const int units = p.num_tiles * p.ksplit;
+    int grid = units < num_sms ? units : num_sms;
     if (grid < 1) return cudaSuccess;
     return launch_pdl(gemm_kernel, dim3(grid), dim3(kGemmThreads), smem, stream, p);
 }

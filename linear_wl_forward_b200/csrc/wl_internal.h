@@ -110,7 +110,9 @@ wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;         // 128 bytes of bf16: one swizzle row
 constexpr int kGemmMaxBN = 256;
-constexpr int kGemmMaxStages = 8;
+constexpr int kGemmMaxStages = 12;
+constexpr int kGemmSwapMaxM = 16;   // swap-AB mode up to this many tokens (measured: at 64 the 128-row x tiles win)
+constexpr int kGemmMaxKSplit = 8;   // K ranges per output tile in swap mode
 constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 
 struct GemmSeg {
@@ -132,6 +134,12 @@ struct GemmParams {
     int nseg;
     int M, K;
     int BN;
+    int swap;         // few-token mode: A = 128-row W0 (or U) tiles, B = x (or T) tiles of mp rows
+    int mp;           // swap: B rows, the token count rounded up to 16 (the MMA's N)
+    int ksplit;       // K-block ranges per output tile (1 unless swap); their sums meet in `part`
+    int kb_split;     // K blocks per range
+    float *part;      // swap, ksplit > 1: [ksplit][tiles][mp][128] partial W0 x sums, then [tiles][mp][128] U T
+    unsigned int *tile_cnt;  // swap, ksplit > 1: per-tile arrival counts, self-resetting (zeroed at allocation)
     int stages;       // pipeline depth (set_gemm_stages)
     int stage_bytes;
     int num_m_tiles;
