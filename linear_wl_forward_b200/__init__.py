@@ -11,7 +11,8 @@ import ctypes
 import os
 
 __all__ = [
-    "WLError", "lib", "linear_forward", "stacked_forward", "decompose",
+    "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
+    "decompose",
     "relative_frobenius_error", "last_device_status", "wait_probe", "PATHS",
     "DECODE_MAX_M", "MAX_RANK", "MAX_PROJ", "STATUS",
 ]
@@ -135,6 +136,43 @@ def stacked_forward(x, projs, ys=None, stream=None, path="auto"):
     _check(lib().wl_forward_ex(xp, M, K, arr, len(projs), PATHS[path], _stream_handle(stream)),
            "wl_forward_ex")
     return ys
+
+
+class PreparedForward:
+    """A stacked forward whose tensors are checked and marshalled once.
+
+    Calling it issues the forward on `stream` (default: torch's current
+    stream) with the same tensors; it returns the list of y_p.  A decode step
+    that runs the same projections on the same buffers every token calls
+    these instead of ``stacked_forward`` and so pays the checks once.  The
+    tensors are kept alive by this object; their storage must not be
+    replaced (in-place writes to x and the weights between calls are fine).
+    """
+
+    def __init__(self, x, projs, ys=None, path="auto"):
+        import torch
+
+        M, K = x.shape
+        if ys is None:
+            ys = [torch.empty(M, W0.shape[0], dtype=torch.bfloat16, device=x.device)
+                  for (W0, _, _, _) in projs]
+        self.ys = ys
+        self._keep = (x, projs, ys)
+        self._arr = (_Proj * len(projs))(*[_make_proj(W0, s, U, V, y, M, K)
+                                           for (W0, s, U, V), y in zip(projs, ys)])
+        self._args = (_dev_ptr(x, torch.bfloat16, "x", (M, K)), M, K, self._arr, len(projs), PATHS[path])
+        self._fn = lib().wl_forward_ex
+
+    def __call__(self, stream=None):
+        xp, M, K, arr, P, path = self._args
+        _check(self._fn(xp, M, K, arr, P, path, _stream_handle(stream)), "wl_forward_ex")
+        return self.ys
+
+
+def prepare_stacked(x, projs, ys=None, path="auto") -> PreparedForward:
+    """``stacked_forward`` with its argument checks done once: returns a
+    callable that issues the forward (see PreparedForward)."""
+    return PreparedForward(x, projs, ys, path)
 
 
 def last_device_status(stream=None) -> int:

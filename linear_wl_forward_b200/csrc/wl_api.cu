@@ -7,7 +7,9 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <memory>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/wl.h"
 #include "wl_internal.h"
@@ -225,13 +227,61 @@ bool build_decode_params(const wl_bf16 *x, int M, int K, const wl_proj *projs, i
 }
 
 // Returns WL_ERR_UNSUPPORTED if the shape cannot take the decode kernel.
+// Decode plans of recent calls, keyed by everything the plan depends on (the
+// call's pointers and sizes).  A decode step issues the same calls with the
+// same buffers every time, so a hit skips the tensor-map encoding and the
+// planning; only the scratch pointers are filled in per call.
+struct DecodeKey {
+    const void *x;
+    int M, K, P;
+    wl_proj projs[kMaxSeg];
+    bool operator==(const DecodeKey &o) const { return std::memcmp(this, &o, sizeof *this) == 0; }
+};
+
+struct DecodeKeyHash {
+    size_t operator()(const DecodeKey &k) const {
+        // FNV-1a over the key's bytes
+        const unsigned char *b = reinterpret_cast<const unsigned char *>(&k);
+        uint64_t h = 1469598103934665603ull;
+        for (size_t i = 0; i < sizeof k; ++i) h = (h ^ b[i]) * 1099511628211ull;
+        return (size_t)h;
+    }
+};
+
+struct DecodeEntry {
+    DecodeParams dp;
+    DecodePlan plan;
+    wl_status status;  // WL_OK or WL_ERR_UNSUPPORTED (the shape cannot take the decode kernel)
+};
+
+constexpr size_t kDecodeCacheMax = 4096;
+std::unordered_map<DecodeKey, std::unique_ptr<DecodeEntry>, DecodeKeyHash> g_decode_cache[kMaxDevices];
+
 wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
                      cudaStream_t stream) {
-    static thread_local DecodeParams dp;  // large (tensor maps); kept off the stack
-    if (!build_decode_params(x, M, K, projs, P, dp)) return WL_OK;
-    DecodePlan plan;
-    wl_status st0 = plan_decode(dp, pool.num_sms, &plan);
-    if (st0 != WL_OK) return st0;
+    DecodeKey key;
+    std::memset(&key, 0, sizeof key);  // padding bytes take part in the comparison
+    key.x = x;
+    key.M = M;
+    key.K = K;
+    key.P = P;
+    std::memcpy(key.projs, projs, sizeof(wl_proj) * P);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WL_ERR_CUDA;
+    auto &cache = g_decode_cache[dev];
+    auto it = cache.find(key);
+    if (it == cache.end()) {
+        if (cache.size() >= kDecodeCacheMax) cache.clear();
+        auto e = std::make_unique<DecodeEntry>();
+        if (!build_decode_params(x, M, K, projs, P, e->dp)) return WL_OK;
+        e->status = plan_decode(e->dp, pool.num_sms, &e->plan);
+        if (e->status != WL_OK && e->status != WL_ERR_UNSUPPORTED) return e->status;
+        it = cache.emplace(key, std::move(e)).first;
+    }
+    DecodeEntry &e = *it->second;
+    if (e.status != WL_OK) return e.status;
+    DecodeParams &dp = e.dp;
+    const DecodePlan &plan = e.plan;
     dp.a.status = pool.words;
     dp.a.sync = reinterpret_cast<unsigned int *>(pool.words + 8);
     if (plan.tpart_bytes) {

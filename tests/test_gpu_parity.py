@@ -170,3 +170,22 @@ def test_gemma4_31b_prefill_sampled_rows():
             if layer == 5 and call.projs[0].family in ("gate", "down"):
                 continue  # MLP shapes already covered by layer 0
             check_call(call, rows=rows)
+
+
+@pytest.mark.gpu
+def test_prepared_matches_stacked():
+    """A prepared call (checks and marshalling done once, then issued twice)
+    gives the same bits as stacked_forward on the same inputs."""
+    import torch
+
+    for M in (1, 12, 40):
+        call = wl_inputs.random_case(31 + M, M, [300, 64], 520, [16, 8], P=2)
+        xd, pd = to_dev(call)
+        ref = [y.cpu() for y in wl.stacked_forward(xd, pd)]
+        prep = wl.prepare_stacked(xd, pd)
+        for _ in range(2):
+            got = [y.cpu() for y in prep()]
+            torch.cuda.synchronize()
+            for a, b in zip(ref, got):
+                assert torch.equal(a, b)
+        assert wl.last_device_status() == 0
