@@ -64,8 +64,10 @@ def _f32(t):
     return t.detach().cpu().contiguous().numpy().astype(np.float32, copy=False)
 
 
-def _run(name, x, W0, s, U, V):
-    lib = _load()
+def _run(name, x, W0, s, U, V, lib=None):
+    """Marshal the operands and call `name` in the oracle library (or in
+    `lib`, a library built from a modified copy of the same source)."""
+    lib = _load() if lib is None else lib
     xb, wb, sb = _bits(x), _bits(W0), _f32(s)
     M, K = xb.shape
     N = wb.shape[0]
