@@ -290,7 +290,41 @@ def secondary_figures(wl, peaks):
         "us_per_call": round(ms * 1e3, 2), "weight_bytes_per_call": b}
     del dev, outs, g
     torch.cuda.empty_cache()
+    out.update(gemma4_layer_figures(wl, peaks))
     out["gemma4_prefill_gate_up_M4096"] = prefill_figure(wl, peaks)
+    return out
+
+
+def gemma4_layer_figures(wl, peaks):
+    """A whole Gemma-4-31B sliding layer (q/k/v stack, o, gate/up stack, down;
+    rank 256) at M = 1 and M = 16 through the library's automatic path choice:
+    two layers of different bands (distinct W0, > L2) in one graph, reported
+    per layer as weight GB/s."""
+    out = {}
+    calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=[0, 12])
+    dev = [to_dev_call(c) for c in calls]
+    layer0 = [c for c in calls if c.layer == 0]
+    wbytes = sum(footprint.call_weight_bytes(p.N, p.K, p.r) for c in layer0 for p in c.projs)
+    for M in (1, 16):
+        xs = {}
+        dev_m, calls_m = [], []
+        for c, dc in zip(calls, dev):
+            K = c.x.shape[1]
+            if K not in xs:
+                xs[K] = wl_inputs.draw_x("gemma4_31b", 4, M, K).cuda()
+            dev_m.append({"x": xs[K], "projs": dc["projs"]})
+            calls_m.append(wl_inputs.Call(c.layer, c.projs, xs[K]))
+        outs, _ = alloc_outputs(calls_m)
+        g = capture(make_step(dev_m, outs, wl), 3)
+        ms = time_graph(g, 5) / 2
+        gbs = wbytes / (ms * 1e-3) / 1e9
+        out[f"gemma4_decode_sliding_layer_M{M}"] = {
+            "GB/s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+            "us_per_layer": round(ms * 1e3, 1), "weight_bytes_per_layer": wbytes,
+            "paths": [call_path(c) for c in calls_m if c.layer == 0]}
+        del outs, g
+    del dev
+    torch.cuda.empty_cache()
     return out
 
 
