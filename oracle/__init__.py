@@ -17,8 +17,8 @@ import subprocess
 
 import numpy as np
 
-from .decompose import (band_of_layer_contiguous, decompose,  # noqa: F401
-                        relative_frobenius_error, theta_reconstruct)
+from .decompose import (band_of_layer_contiguous, decompose, decompose_als,  # noqa: F401
+                        relative_frobenius_error, theta_objective, theta_reconstruct)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "wl_oracle.c")

@@ -96,3 +96,57 @@ def test_explicit_interleaved_bands():
     W0, s, U, V = oracle.decompose(W, G=2, r=1, band_of_layer=[0, 1, 0, 1])
     assert np.allclose(W0[0], (W[0] + W[2]) / 2)
     assert np.allclose(W0[1], (W[1] + W[3]) / 2)
+
+
+# ------------------------------------------------------------- ALS refinement --
+@pytest.mark.parametrize("G,r,bands", [(1, 0, None), (1, 3, None), (2, 2, None), (2, 1, [0, 1, 1, 0])])
+def test_als_objective_never_increases(G, r, bands):
+    """Every ALS step is an exact least-squares minimisation over its block of
+    unknowns, so the total squared residual cannot grow at any step."""
+    W = rand_w(20 + G + r, 4, 7, 9)
+    trace = []
+    oracle.decompose_als(W, G, r, iters=6, band_of_layer=bands, trace=trace)
+    for a, b in zip(trace, trace[1:]):
+        assert b <= a * (1 + 1e-12) + 1e-12
+
+
+def test_als_zero_iterations_is_the_mean_start():
+    W = rand_w(21, 3, 6, 5)
+    a = oracle.decompose(W, G=1, r=2)
+    b = oracle.decompose_als(W, G=1, r=2, iters=0)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_als_rank0_converges_to_best_rank1_per_row():
+    """With r = 0 and one band the objective separates over rows: row n of all
+    layers is an L x K matrix M_n fitted by s[:, n] W0[n]^T, a rank-1 model,
+    and ALS is an alternating power iteration.  It must reach the Eckart-Young
+    optimum sum_n sum_{i >= 2} sigma_i(M_n)^2 (numpy's SVD of each M_n)."""
+    W = rand_w(22, 4, 5, 6)
+    trace = []
+    oracle.decompose_als(W, G=1, r=0, iters=300, trace=trace)
+    best = sum(float(np.sum(np.linalg.svd(W[:, n, :], compute_uv=False)[1:] ** 2)) for n in range(W.shape[1]))
+    assert abs(trace[-1] - best) <= 1e-9 * best
+    assert trace[0] > best * (1 + 1e-3)  # the mean start is not already optimal
+
+
+def test_als_hand_example_two_layers():
+    """W_1 = [2, 0], W_2 = [0, 1] (one row, one band, r = 0): the stacked 2 x 2
+    matrix has singular values 2 and 1, so ALS must approach a residual of
+    1^2 = 1 with W0 along [1, 0] and the second layer's scale -> 0; the mean
+    start (W0 = [1, 0.5]) has residual 1.6."""
+    W = np.array([[[2.0, 0.0]], [[0.0, 1.0]]])
+    trace = []
+    W0, s, U, V = oracle.decompose_als(W, G=1, r=0, iters=60, trace=trace)
+    assert trace[0] == pytest.approx(1.6, abs=1e-12)
+    assert trace[-1] == pytest.approx(1.0, abs=1e-12)
+    assert abs(W0[0, 0, 1]) <= 1e-12 * abs(W0[0, 0, 0])
+    assert abs(s[1, 0]) <= 1e-12
+
+
+def test_als_keeps_passthrough_exact():
+    W = rand_w(23, 3, 5, 7)
+    W0, s, U, V = oracle.decompose_als(W, G=3, r=2, iters=3)
+    for l in range(3):
+        assert oracle.relative_frobenius_error(W[l], W0[l], s[l], U[l], V[l]) <= 1e-15
