@@ -176,6 +176,23 @@ wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r,
                        const int *band_of_layer, float *W0, float *s, float *U,
                        float *V, double *rel_err);
 
+/* wl_decompose followed by `iters` rounds of alternating least squares over
+ * the band-mean start ("Quality (Gemma 4 31B)", "ALS optimization barely
+ * helps": ALS tried as an improvement over the mean W0; the pages name the
+ * method, not its steps).  One round makes three exact least-squares updates
+ * of the total squared residual sum_l ||W_l - diag(s_l) W0 - U_l V_l^T||_F^2,
+ * each over its own unknowns with the others fixed:
+ *   1. W0_b[n] = sum_{l in b} s_l[n] (W_l[n] - (U_l V_l^T)[n]) / sum_{l in b} s_l[n]^2
+ *      (the row is kept when every s_l[n] of the band is 0);
+ *   2. s_l[n] = <W_l[n] - (U_l V_l^T)[n], W0_b[n]> / ||W0_b[n]||^2 (1 for a zero row);
+ *   3. U_l V_l^T = rank-r truncated SVD of W_l - diag(s_l) W0_b.
+ * So the total residual never grows.  iters = 0 is wl_decompose.  Same
+ * arguments, layouts, outputs and errors as wl_decompose (iters < 0 is
+ * WL_ERR_INVALID_ARG); the factors are carried in fp64 between rounds. */
+wl_status wl_decompose_als(const float *W, int L, int N, int K, int G, int r,
+                           const int *band_of_layer, int iters, float *W0, float *s,
+                           float *U, float *V, double *rel_err);
+
 /* ||W - (diag(s) W0 + U V^T)||_F / ||W||_F for one layer, host pointers, fp64
  * ("Quality": relative Frobenius error of diag(s).W0 + U.V^T against the true
  * weight).  Returns a negative value for invalid arguments. */

@@ -57,6 +57,7 @@ def lib():
         L.wl_stacked_forward.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, vp]
         L.wl_forward_ex.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, ci, vp]
         L.wl_decompose.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp]
+        L.wl_decompose_als.argtypes = [vp, ci, ci, ci, ci, ci, vp, ci, vp, vp, vp, vp, vp]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
         L.wl_relative_frobenius_error.restype = ctypes.c_double
         L.wl_status_string.argtypes = [ci]
@@ -64,7 +65,7 @@ def lib():
         L.wl_last_device_status.argtypes = [vp]
         L.wl_wait_probe.argtypes = [cll, vp]
         L.wl_version.restype = ci
-        for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose",
+        for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose", "wl_decompose_als",
                      "wl_last_device_status", "wl_wait_probe"):
             getattr(L, name).restype = ci
         _lib = L
@@ -184,9 +185,11 @@ def wait_probe(limit_ns: int, stream=None):
     _check(lib().wl_wait_probe(int(limit_ns), _stream_handle(stream)), "wl_wait_probe")
 
 
-def decompose(W, G: int, r: int, band_of_layer=None):
-    """Host decomposition (include/wl.h, wl_decompose).  W: (L, N, K) float32
-    numpy array.  Returns (W0 (G,N,K), s (L,N), U (L,N,r), V (L,K,r), rel_err (L,))."""
+def decompose(W, G: int, r: int, band_of_layer=None, als_iters: int = 0):
+    """Host decomposition (include/wl.h, wl_decompose; with als_iters > 0,
+    wl_decompose_als: that many alternating-least-squares rounds over the
+    band-mean start).  W: (L, N, K) float32 numpy array.  Returns
+    (W0 (G,N,K), s (L,N), U (L,N,r), V (L,K,r), rel_err (L,))."""
     import numpy as np
 
     W = np.ascontiguousarray(W, dtype=np.float32)
@@ -199,10 +202,15 @@ def decompose(W, G: int, r: int, band_of_layer=None):
     bands = None
     if band_of_layer is not None:
         bands = np.ascontiguousarray(band_of_layer, dtype=np.int32)
-    _check(lib().wl_decompose(W.ctypes.data, L, N, K, G, r,
-                              None if bands is None else bands.ctypes.data, W0.ctypes.data,
-                              s.ctypes.data, U.ctypes.data, V.ctypes.data, err.ctypes.data),
-           "wl_decompose")
+    bp = None if bands is None else bands.ctypes.data
+    if als_iters:
+        _check(lib().wl_decompose_als(W.ctypes.data, L, N, K, G, r, bp, int(als_iters), W0.ctypes.data,
+                                      s.ctypes.data, U.ctypes.data, V.ctypes.data, err.ctypes.data),
+               "wl_decompose_als")
+    else:
+        _check(lib().wl_decompose(W.ctypes.data, L, N, K, G, r, bp, W0.ctypes.data,
+                                  s.ctypes.data, U.ctypes.data, V.ctypes.data, err.ctypes.data),
+               "wl_decompose")
     return W0, s, U, V, err
 
 

@@ -61,9 +61,9 @@ void jacobi_orthogonalize(std::vector<double> &A, int m, int n, std::vector<doub
 }
 
 // Rank-r truncated SVD of R (N x K, row-major): U = P_r S_r (N x r), V = Q_r (K x r).
-void truncated_svd(const std::vector<double> &R, int N, int K, int r, float *U, float *V) {
-    std::memset(U, 0, sizeof(float) * (size_t)N * r);
-    std::memset(V, 0, sizeof(float) * (size_t)K * r);
+void truncated_svd(const std::vector<double> &R, int N, int K, int r, double *U, double *V) {
+    std::fill(U, U + (size_t)N * r, 0.0);
+    std::fill(V, V + (size_t)K * r, 0.0);
     if (r == 0) return;
     const bool cols_are_k = K <= N;  // orthogonalise the K columns of R, else the N columns of R^T
     const int m = cols_are_k ? N : K, n = cols_are_k ? K : N;
@@ -95,12 +95,12 @@ void truncated_svd(const std::vector<double> &R, int N, int K, int r, float *U, 
         const double *q = &Q[(size_t)i * n];
         if (cols_are_k) {
             // R Q = A: column i of A is sigma_i p_i (length N); Q column is v_i (length K)
-            for (int a = 0; a < N; ++a) U[(size_t)a * r + c] = (float)col[a];
-            for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = (float)q[b];
+            for (int a = 0; a < N; ++a) U[(size_t)a * r + c] = col[a];
+            for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = q[b];
         } else {
             // R^T Q = A: R = Q A^T; left vectors are Q columns (length N), right A/sigma (length K)
-            for (int a = 0; a < N; ++a) U[(size_t)a * r + c] = (float)(q[a] * sg);
-            for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = (float)(col[b] / sg);
+            for (int a = 0; a < N; ++a) U[(size_t)a * r + c] = q[a] * sg;
+            for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = col[b] / sg;
         }
     }
 }
@@ -120,14 +120,24 @@ double rel_err_fp64(const float *W, const float *W0, const float *s, const float
     return den > 0 ? std::sqrt(num / den) : std::sqrt(num);
 }
 
-}  // namespace
+// Row n of U_l V_l^T (fp64 factors) into out[K].
+void uv_row(const double *Ul, const double *Vl, int n, int K, int r, double *out) {
+    for (int k = 0; k < K; ++k) {
+        double acc = 0;
+        for (int j = 0; j < r; ++j) acc += Ul[(size_t)n * r + j] * Vl[(size_t)k * r + j];
+        out[k] = acc;
+    }
+}
 
-extern "C" {
-
-wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r, const int *band_of_layer,
-                       float *W0, float *s, float *U, float *V, double *rel_err) {
+// Band-mean start, then `iters` alternating least-squares iterations ("Quality
+// (Gemma 4 31B)", "ALS optimization barely helps"), each of three exact
+// block updates of the total squared residual: every band's W0 with s and
+// U V^T fixed, every s with W0 and U V^T fixed, every U V^T (truncated SVD of
+// W_l - diag(s_l) W0) with W0 and s fixed.
+wl_status decompose_impl(const float *W, int L, int N, int K, int G, int r, const int *band_of_layer, int iters,
+                         float *W0, float *s, float *U, float *V, double *rel_err) {
     if (!W || !W0 || !s || (r > 0 && (!U || !V))) return WL_ERR_INVALID_ARG;
-    if (L < 1 || N < 1 || K < 1 || G < 1 || r < 0) return WL_ERR_INVALID_ARG;
+    if (L < 1 || N < 1 || K < 1 || G < 1 || r < 0 || iters < 0) return WL_ERR_INVALID_ARG;
     try {
         std::vector<int> band(L);
         for (int l = 0; l < L; ++l) {
@@ -143,38 +153,92 @@ wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r, const 
             const float *src = W + (size_t)l * NK;
             for (size_t i = 0; i < NK; ++i) dst[i] += src[i];
         }
-        for (int b = 0; b < G; ++b) {
-            double *dst = &w0[(size_t)b * NK];
+        for (int b = 0; b < G; ++b)
             if (count[b] > 0)
-                for (size_t i = 0; i < NK; ++i) dst[i] /= count[b];
-            for (size_t i = 0; i < NK; ++i) W0[(size_t)b * NK + i] = (float)dst[i];
-        }
-        std::vector<double> R(NK);
-        for (int l = 0; l < L; ++l) {
+                for (size_t i = 0; i < NK; ++i) w0[(size_t)b * NK + i] /= count[b];
+        std::vector<double> sd((size_t)L * N, 1.0);
+        std::vector<double> Ud((size_t)L * N * r, 0.0), Vd((size_t)L * K * r, 0.0);
+        std::vector<double> R(NK), uv(K);
+        // s_l[n] = <W_l[n] - (U_l V_l^T)[n], W0_b[n]> / ||W0_b[n]||^2 (1 for a zero row)
+        auto fit_scales = [&](int l, bool with_uv) {
             const float *w = W + (size_t)l * NK;
             const double *b0 = &w0[(size_t)band[l] * NK];
-            float *sl = s + (size_t)l * N;
             for (int n = 0; n < N; ++n) {
+                if (with_uv && r > 0) uv_row(&Ud[(size_t)l * N * r], &Vd[(size_t)l * K * r], n, K, r, uv.data());
                 double num = 0, den = 0;
                 for (int k = 0; k < K; ++k) {
-                    num += (double)w[(size_t)n * K + k] * b0[(size_t)n * K + k];
+                    const double t = (double)w[(size_t)n * K + k] - (with_uv && r > 0 ? uv[k] : 0.0);
+                    num += t * b0[(size_t)n * K + k];
                     den += b0[(size_t)n * K + k] * b0[(size_t)n * K + k];
                 }
-                const double sc = den > 0 ? num / den : 1.0;
-                sl[n] = (float)sc;
-                for (int k = 0; k < K; ++k)
-                    R[(size_t)n * K + k] = (double)w[(size_t)n * K + k] - sc * b0[(size_t)n * K + k];
+                sd[(size_t)l * N + n] = den > 0 ? num / den : 1.0;
             }
-            float *Ul = r > 0 ? U + (size_t)l * N * r : nullptr;
-            float *Vl = r > 0 ? V + (size_t)l * K * r : nullptr;
-            if (r > 0) truncated_svd(R, N, K, r, Ul, Vl);
-            if (rel_err)
-                rel_err[l] = rel_err_fp64(w, W0 + (size_t)band[l] * NK, sl, Ul, Vl, N, K, r);
+        };
+        // U_l V_l^T = rank-r truncated SVD of W_l - diag(s_l) W0_b
+        auto fit_delta = [&](int l) {
+            if (r == 0) return;
+            const float *w = W + (size_t)l * NK;
+            const double *b0 = &w0[(size_t)band[l] * NK];
+            for (int n = 0; n < N; ++n)
+                for (int k = 0; k < K; ++k)
+                    R[(size_t)n * K + k] = (double)w[(size_t)n * K + k] - sd[(size_t)l * N + n] * b0[(size_t)n * K + k];
+            truncated_svd(R, N, K, r, &Ud[(size_t)l * N * r], &Vd[(size_t)l * K * r]);
+        };
+        for (int l = 0; l < L; ++l) {
+            fit_scales(l, false);
+            fit_delta(l);
         }
+        std::vector<double> num(K);
+        for (int it = 0; it < iters; ++it) {
+            // W0_b[n] = sum_l s_l[n] (W_l[n] - (U_l V_l^T)[n]) / sum_l s_l[n]^2 (kept if all s are 0)
+            for (int b = 0; b < G; ++b) {
+                for (int n = 0; n < N; ++n) {
+                    std::fill(num.begin(), num.end(), 0.0);
+                    double den = 0;
+                    for (int l = 0; l < L; ++l) {
+                        if (band[l] != b) continue;
+                        const double sc = sd[(size_t)l * N + n];
+                        const float *w = W + (size_t)l * NK + (size_t)n * K;
+                        if (r > 0) uv_row(&Ud[(size_t)l * N * r], &Vd[(size_t)l * K * r], n, K, r, uv.data());
+                        for (int k = 0; k < K; ++k) num[k] += sc * ((double)w[k] - (r > 0 ? uv[k] : 0.0));
+                        den += sc * sc;
+                    }
+                    if (den > 0)
+                        for (int k = 0; k < K; ++k) w0[(size_t)b * NK + (size_t)n * K + k] = num[k] / den;
+                }
+            }
+            for (int l = 0; l < L; ++l) fit_scales(l, true);
+            for (int l = 0; l < L; ++l) fit_delta(l);
+        }
+        for (size_t i = 0; i < (size_t)G * NK; ++i) W0[i] = (float)w0[i];
+        for (size_t i = 0; i < (size_t)L * N; ++i) s[i] = (float)sd[i];
+        if (r > 0) {
+            for (size_t i = 0; i < Ud.size(); ++i) U[i] = (float)Ud[i];
+            for (size_t i = 0; i < Vd.size(); ++i) V[i] = (float)Vd[i];
+        }
+        if (rel_err)
+            for (int l = 0; l < L; ++l)
+                rel_err[l] = rel_err_fp64(W + (size_t)l * NK, W0 + (size_t)band[l] * NK, s + (size_t)l * N,
+                                          r > 0 ? U + (size_t)l * N * r : nullptr,
+                                          r > 0 ? V + (size_t)l * K * r : nullptr, N, K, r);
     } catch (const std::bad_alloc &) {
         return WL_ERR_NOMEM;
     }
     return WL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r, const int *band_of_layer,
+                       float *W0, float *s, float *U, float *V, double *rel_err) {
+    return decompose_impl(W, L, N, K, G, r, band_of_layer, 0, W0, s, U, V, rel_err);
+}
+
+wl_status wl_decompose_als(const float *W, int L, int N, int K, int G, int r, const int *band_of_layer,
+                           int iters, float *W0, float *s, float *U, float *V, double *rel_err) {
+    return decompose_impl(W, L, N, K, G, r, band_of_layer, iters, W0, s, U, V, rel_err);
 }
 
 double wl_relative_frobenius_error(const float *W, const float *W0, const float *s, const float *U,

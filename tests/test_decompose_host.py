@@ -59,3 +59,40 @@ def test_error_non_increasing_in_rank():
         assert err.mean() <= prev + 1e-6
         prev = err.mean()
     assert prev < 1e-5
+
+
+@pytest.mark.parametrize("L,N,K,G,r,iters,bands", [(4, 12, 20, 2, 3, 3, None), (3, 9, 14, 1, 0, 5, None),
+                                                   (4, 10, 8, 2, 2, 2, [0, 1, 1, 0]), (2, 6, 6, 1, 4, 4, None)])
+def test_als_matches_oracle(L, N, K, G, r, iters, bands):
+    """wl_decompose_als against the numpy ALS oracle: W0, s, U V^T and the
+    errors after the same number of rounds."""
+    W = np.random.default_rng(L * 1000 + N * 10 + K + iters).standard_normal((L, N, K)).astype(np.float32)
+    W0, s, U, V, err = wl.decompose(W, G, r, band_of_layer=bands, als_iters=iters)
+    oW0, os_, oU, oV = oracle.decompose_als(W.astype(np.float64), G, r, iters, band_of_layer=bands)
+    b = oracle.band_of_layer_contiguous(L, G) if bands is None else bands
+    assert np.allclose(W0, oW0, atol=1e-5, rtol=1e-5)
+    assert np.allclose(s, os_, atol=1e-5, rtol=1e-5)
+    for l in range(L):
+        uv = U[l].astype(np.float64) @ V[l].astype(np.float64).T
+        ouv = oU[l] @ oV[l].T
+        assert np.max(np.abs(uv - ouv)) <= 1e-4 * max(1.0, np.max(np.abs(ouv)))
+        oe = oracle.relative_frobenius_error(W[l], oW0[b[l]], os_[l], oU[l], oV[l])
+        assert abs(err[l] - oe) < 1e-5
+
+
+def test_als_zero_rounds_is_plain_decompose_and_rounds_do_not_hurt():
+    W = np.random.default_rng(9).standard_normal((4, 10, 12)).astype(np.float32)
+    a = wl.decompose(W, 1, 2)
+    b = wl.decompose(W, 1, 2, als_iters=0)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+    c = wl.decompose(W, 1, 2, als_iters=4)
+    # the total squared residual can only go down; per layer it may move either way
+    total = lambda e: float(np.sum(e ** 2 * np.sum(W.astype(np.float64) ** 2, axis=(1, 2))))
+    assert total(c[4]) <= total(a[4]) * (1 + 1e-6)
+
+
+def test_als_rejects_negative_rounds():
+    W = np.zeros((2, 3, 4), np.float32)
+    with pytest.raises(wl.WLError):
+        wl.decompose(W, 1, 1, als_iters=-1)
