@@ -275,8 +275,8 @@ def traffic_from_profile(kernel, call):
 
 
 # -------------------------------------------------------------- secondary --
-def secondary_figures(wl, peaks):
-    out = {}
+def secondary_figures(wl, peaks, headline_ms):
+    out = {"gemma3_decode_dense_comparator": dense_figure(wl, peaks, headline_ms)}
     # Gemma-4-31B decode, M = 1: stacked gate/up of two bands (rotating, > L2)
     calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=[0, 12], families=("gate",))
     dev = [to_dev_call(c) for c in calls]
@@ -293,6 +293,36 @@ def secondary_figures(wl, peaks):
     out.update(gemma4_layer_figures(wl, peaks))
     out["gemma4_prefill_gate_up_M4096"] = prefill_figure(wl, peaks)
     return out
+
+
+def dense_figure(wl, peaks, headline_ms):
+    """The dense comparator of the Gemma-3-1B decode sweep: every projection's
+    W_eff = diag(s) W0 + U V^T rebuilt once on the GPU (wl.materialize_weight),
+    then the same 26-layer sweep as a plain rank-0 forward over the 26 distinct
+    dense weights.  Reported against the weightless sweep's time per step."""
+    calls = wl_inputs.gemma3_sweep(seed=2, G=13, r=16, M=1)
+    dev = []
+    wbytes = 0
+    for c in calls:
+        dc = to_dev_call(c)
+        projs = []
+        for (W0, s, U, V), p in zip(dc["projs"], c.projs):
+            Weff = wl.materialize_weight(W0, s, U, V)
+            projs.append((Weff, torch.ones(p.N, device="cuda"), None, None))
+            wbytes += p.N * p.K * 2 + p.N * 4
+        dev.append({"x": dc["x"], "projs": projs})
+        del dc
+    torch.cuda.synchronize()
+    assert wl.last_device_status() == 0
+    outs, _ = alloc_outputs(calls)
+    g = capture(make_step(dev, outs, wl), 3)
+    ms = time_graph(g, 50)
+    del dev, outs, g
+    torch.cuda.empty_cache()
+    gbs = wbytes / (ms * 1e-3) / 1e9
+    return {"ms_per_step": round(ms, 4), "GB/s": round(gbs, 1),
+            "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "weight_bytes_per_step": wbytes,
+            "weightless_over_dense_time": round(headline_ms / ms, 4)}
 
 
 def gemma4_layer_figures(wl, peaks):
@@ -553,7 +583,7 @@ def main():
     if rank == 0 and world == 1:
         line["roofline"] = decode_roofline(wl, peaks)
         if not args.no_secondary:
-            line["secondary"] = secondary_figures(wl, peaks)
+            line["secondary"] = secondary_figures(wl, peaks, ms_step)
         b, s, n = oracle_sample(calls, budget_s=12.0)
         line["cpu_baseline"] = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": 1,
                                 "kind": "oracle",

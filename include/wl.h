@@ -199,6 +199,21 @@ wl_status wl_decompose_als(const float *W, int L, int N, int K, int G, int r,
 double wl_relative_frobenius_error(const float *W, const float *W0, const float *s,
                                    const float *U, const float *V, int N, int K, int r);
 
+/* W_eff = diag(s) W0 + U V^T: the dense weight a theta bundle stands for,
+ * rebuilt once so later calls can run the plain dense product ("Add a new
+ * model architecture", "Override the graph build", step 5: the
+ * precompute-outside path).  A dense forward is then wl_linear_forward with
+ * W0 = W_eff, s = 1 and r = 0.
+ *   W0 : device, N x K bf16 row-major       s : device, N fp32
+ *   U  : device, N x r bf16 row-major       V : device, K x r bf16 row-major
+ *   W_eff : device, N x K bf16 row-major (written; must not overlap the inputs)
+ * fp32 accumulation, one rounding to bf16.  N, K, r >= 0 (N or K == 0 is a
+ * no-op), r <= WL_MAX_RANK; U and V may be NULL iff r == 0.  Asynchronous on
+ * `stream`.  Returns WL_ERR_INVALID_ARG for null pointers or negative sizes. */
+wl_status wl_materialize_weight(const wl_bf16 *W0, const float *s, const wl_bf16 *U,
+                                const wl_bf16 *V, wl_bf16 *W_eff, int N, int K, int r,
+                                void *stream);
+
 /* Static description of a status code. */
 const char *wl_status_string(wl_status status);
 

@@ -12,6 +12,7 @@ import os
 
 __all__ = [
     "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
+    "materialize_weight",
     "decompose",
     "relative_frobenius_error", "last_device_status", "wait_probe", "PATHS",
     "DECODE_MAX_M", "MAX_RANK", "MAX_PROJ", "STATUS",
@@ -58,6 +59,7 @@ def lib():
         L.wl_forward_ex.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, ci, vp]
         L.wl_decompose.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp]
         L.wl_decompose_als.argtypes = [vp, ci, ci, ci, ci, ci, vp, ci, vp, vp, vp, vp, vp]
+        L.wl_materialize_weight.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, vp]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
         L.wl_relative_frobenius_error.restype = ctypes.c_double
         L.wl_status_string.argtypes = [ci]
@@ -66,6 +68,7 @@ def lib():
         L.wl_wait_probe.argtypes = [cll, vp]
         L.wl_version.restype = ci
         for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose", "wl_decompose_als",
+                     "wl_materialize_weight",
                      "wl_last_device_status", "wl_wait_probe"):
             getattr(L, name).restype = ci
         _lib = L
@@ -174,6 +177,25 @@ def prepare_stacked(x, projs, ys=None, path="auto") -> PreparedForward:
     """``stacked_forward`` with its argument checks done once: returns a
     callable that issues the forward (see PreparedForward)."""
     return PreparedForward(x, projs, ys, path)
+
+
+def materialize_weight(W0, s, U, V, out=None, stream=None):
+    """W_eff = diag(s) W0 + U V^T (N x K bf16) on the GPU: the dense weight the
+    bundle stands for, for the precompute-outside path (a dense forward is
+    then ``linear_forward(x, W_eff, ones, None, None)``)."""
+    import torch
+
+    N, K = W0.shape
+    r = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.bfloat16, device=W0.device)
+    _check(lib().wl_materialize_weight(
+        _dev_ptr(W0, torch.bfloat16, "W0", (N, K)), _dev_ptr(s, torch.float32, "s", (N,)),
+        _dev_ptr(U, torch.bfloat16, "U", (N, r)) if r else None,
+        _dev_ptr(V, torch.bfloat16, "V", (K, r)) if r else None,
+        _dev_ptr(out, torch.bfloat16, "out", (N, K)), N, K, r, _stream_handle(stream)),
+        "wl_materialize_weight")
+    return out
 
 
 def last_device_status(stream=None) -> int:

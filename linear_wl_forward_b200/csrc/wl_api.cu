@@ -524,6 +524,22 @@ const char *wl_status_string(wl_status s) {
     return "unknown status";
 }
 
+wl_status wl_materialize_weight(const wl_bf16 *W0, const float *s, const wl_bf16 *U, const wl_bf16 *V,
+                                wl_bf16 *W_eff, int N, int K, int r, void *stream) {
+    if (N < 0 || K < 0 || r < 0) return WL_ERR_INVALID_ARG;
+    if (r > WL_MAX_RANK) return WL_ERR_UNSUPPORTED;
+    if (N == 0 || K == 0) return WL_OK;
+    if (!W0 || !s || !W_eff || (r > 0 && (!U || !V))) return WL_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(wl::g_mu);
+    wl::DevicePool *pool = nullptr;
+    wl_status st = wl::pool_for_current_device(&pool);
+    if (st != WL_OK) return st;
+    return wl::from_cuda(wl::launch_materialize(
+        reinterpret_cast<const __nv_bfloat16 *>(W0), s, reinterpret_cast<const __nv_bfloat16 *>(U),
+        reinterpret_cast<const __nv_bfloat16 *>(V), reinterpret_cast<__nv_bfloat16 *>(W_eff), N, K, r,
+        static_cast<cudaStream_t>(stream)));
+}
+
 wl_status wl_last_device_status(void *stream) {
     std::lock_guard<std::mutex> lock(wl::g_mu);
     wl::DevicePool *pool = nullptr;

@@ -168,6 +168,12 @@ cudaError_t launch_transpose_v(const TransposeVArgs &a, cudaStream_t stream);
 cudaError_t launch_pad_u(const __nv_bfloat16 *U, int N, int r, int r_pad,
                          __nv_bfloat16 *Upad, cudaStream_t stream);
 
+// ---------------------------------------------------------- materialize ----
+// Weff = diag(s) W0 + U V^T (bf16 out, fp32 accumulation), all N x K row-major.
+cudaError_t launch_materialize(const __nv_bfloat16 *W0, const float *s, const __nv_bfloat16 *U,
+                               const __nv_bfloat16 *V, __nv_bfloat16 *Weff, int N, int K, int r,
+                               cudaStream_t stream);
+
 // --------------------------------------------------------------- probes ----
 cudaError_t launch_wait_probe(int *flag, int *status, unsigned long long limit_ns,
                               cudaStream_t stream);
