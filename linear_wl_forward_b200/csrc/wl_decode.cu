@@ -68,6 +68,7 @@ constexpr int NTH = kDecodeThreads;
 constexpr int BR = kDecodeBlockRows;
 constexpr int CK = kDecodeChunkK;
 constexpr size_t kLocalVBytes = 96 * 1024;    // local T when each CTA's V is at most this
+constexpr size_t kFusedLocalVBytes = 136 * 1024;  // the same for fused local T and at most two blocks a CTA
 constexpr uint32_t kDecodeMaxSmem = 227 * 1024;
 constexpr uint32_t kSmallSmem = 110 * 1024;   // two CTAs per SM
 constexpr size_t kSmallCtaBytes = 256 * 1024; // W0 + U per CTA up to which a call is small
@@ -361,6 +362,15 @@ __device__ __forceinline__ void w0_chunk(float (&acc)[NT][4], uint32_t cbase, co
             for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], a[kq], bx[kq][nt][0], bx[kq][nt][1]);
 }
 
+// w0_chunk plus, on the same x fragments, the chunk's share of T = V^T x for
+// the rank r <= 32 of the CTA's projection (fused local T): A = V^T from the
+// staged V rows (row k at k * r) through ldmatrix.trans, rows past K masked.
+template <int NT, int FT, bool FULL>
+__device__ __forceinline__ void w0v_chunk(float (&acc)[NT][4], float (&acct)[FT][NT][4], uint32_t cbase,
+                                          const uint32_t (&swz)[CK / 16], int kk0, int K,
+                                          const bool (&nvalid)[NT], const uint32_t (&xs_lane)[NT],
+                                          uint32_t v_lane, int r, int q);
+
 // One 16 x 64 chunk of U times T (columns j0 .. j0+63 of the rank r).
 template <int NT>
 __device__ __forceinline__ void u_chunk(float (&acu)[NT][4], uint32_t cbase, const uint32_t (&swz)[CK / 16],
@@ -457,6 +467,51 @@ __device__ __forceinline__ void vt_frag(uint32_t (&a)[4], uint32_t v_lane, int r
     if (kb + 16 > k1) {
         if (kb + 2 * q >= k1) a[0] = a[1] = 0u;
         if (kb + 8 + 2 * q >= k1) a[2] = a[3] = 0u;
+    }
+}
+
+template <int NT, int FT, bool FULL>
+__device__ __forceinline__ void w0v_chunk(float (&acc)[NT][4], float (&acct)[FT][NT][4], uint32_t cbase,
+                                          const uint32_t (&swz)[CK / 16], int kk0, int K,
+                                          const bool (&nvalid)[NT], const uint32_t (&xs_lane)[NT],
+                                          uint32_t v_lane, int r, int q) {
+    // two k-steps at a time: the fused variant runs under the compact
+    // variant's register limit
+#pragma unroll
+    for (int kh = 0; kh < CK / 32; ++kh) {
+        uint32_t a[2][4];
+        uint32_t bx[2][NT][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int kq = kh * 2 + h, kk = kk0 + kq * 16;
+            const bool step = FULL || kk < K;
+            const bool hi_ok = FULL || kk + 8 < K;
+            if (step) ldmatrix_x4(cbase + swz[kq], a[h]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                uint32_t b0 = 0u, b1 = 0u;
+                if (step && nvalid[nt]) {
+                    b0 = lds32(xs_lane[nt] + (uint32_t)kk * 2u);
+                    if (hi_ok) b1 = lds32(xs_lane[nt] + (uint32_t)kk * 2u + 16u);
+                }
+                bx[h][nt][0] = b0;
+                bx[h][nt][1] = b1;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int kk = kk0 + (kh * 2 + h) * 16;
+            if (!(FULL || kk < K)) continue;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(acc[nt], a[h], bx[h][nt][0], bx[h][nt][1]);
+#pragma unroll
+            for (int jt = 0; jt < FT; ++jt) {
+                uint32_t av[4];
+                vt_frag(av, v_lane, r, 0, kk, K, jt * 16, q);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(acct[jt][nt], av, bx[h][nt][0], bx[h][nt][1]);
+            }
+        }
     }
 }
 
@@ -774,7 +829,7 @@ __device__ __forceinline__ void step_scales(const DecodeArgs &p, const Step &S, 
 
 }  // namespace
 
-template <int NT, bool XS, bool SMALL>
+template <int NT, bool XS, bool SMALL, int FT>
 __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid_constant__ DecodeParams P) {
     // The next kernel in the stream may launch now; it waits for this grid
     // before it reads anything this grid writes.
@@ -956,7 +1011,18 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     bool ok = true;
     if (p.t_mode != kTNone && p.v_stage)
         ok = !__syncthreads_or(!mbar_wait(vbar, 0, p.status, p.timeout_ns) || *abort_flag != 0);
-    if (ok && p.t_mode == kTLocal) form_t_local<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red, Ts);
+    // Fused local T (FT > 0: a variant of its own, launched for t_fused with
+    // FT 16-column tiles of the rank): the one projection with a delta that
+    // this CTA's rows touch; its V rows open the staged region.
+    constexpr bool fused = FT > 0;
+    int t_sp = -1;
+    if (fused)
+        for (int sp = 0; sp < p.nseg && t_sp < 0; ++sp)
+            if (seg_touched(p.seg[sp], blk_lo, blk_hi)) t_sp = sp;
+    // fused: the epilogues read the staged U rows from the first step on
+    if (ok && fused && p.u_stage)
+        ok = !__syncthreads_or(!mbar_wait(ubar, 0, p.status, p.timeout_ns) || *abort_flag != 0);
+    if (ok && p.t_mode == kTLocal && !fused) form_t_local<NT, XS>(p, blk_lo, blk_hi, xsrc, xld, vs, red, Ts);
 
 
     const int g = lane >> 2, q = lane & 3;          // fragment row / column-pair index
@@ -977,6 +1043,15 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
         xs_lane[nt] = smem_addr(xs) + (uint32_t)((nn * p.x_ld + 2 * q) * 2);
         xg_lane[nt] = p.x + (size_t)nn * K + 2 * q;
     }
+    // Fused local T: the warp's partial sums over its K chunks.
+    constexpr int FTA = FT > 0 ? FT : 1;
+    float acct[FTA][NT][4];
+#pragma unroll
+    for (int jt = 0; jt < FTA; ++jt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acct[jt][nt][e] = 0.f;
 
     bool u_ready = false;  // the staged U rows have been waited for
     uint32_t consumed = 0;
@@ -1032,6 +1107,30 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
                 z += f[fe];
                 d += f[4 + fe];
             }
+            if (fused && Su.has_w && Su.rw > 0 && row < Su.bw.nrows) {
+                // U T of this output: the staged U row times token n's T slice
+                const DecodeSeg &sg = p.seg[Su.bw.sp];
+                int b0, b1;
+                seg_block_range(sg, blk_lo, blk_hi, b0, b1);
+                const __nv_bfloat16 *ur = reinterpret_cast<const __nv_bfloat16 *>(
+                                              us + u_stage_off(p, Su.bw.sp, blk_lo, blk_hi)) +
+                                          (size_t)(Su.bw.row0 - (b0 - sg.blk_begin) * BR + row) * Su.rw;
+                const float *tr = Ts + (size_t)n * p.t_ld + sg.t_off;
+                d = 0.f;
+                for (int j = 0; j < Su.rw; j += 8) {
+                    const uint4 uv = *reinterpret_cast<const uint4 *>(ur + j);
+                    const float4 ta = *reinterpret_cast<const float4 *>(tr + j);
+                    const float4 tb = *reinterpret_cast<const float4 *>(tr + j + 4);
+                    d = fmaf(bf16lo(uv.x), ta.x, d);
+                    d = fmaf(bf16hi(uv.x), ta.y, d);
+                    d = fmaf(bf16lo(uv.y), ta.z, d);
+                    d = fmaf(bf16hi(uv.y), ta.w, d);
+                    d = fmaf(bf16lo(uv.z), tb.x, d);
+                    d = fmaf(bf16hi(uv.z), tb.y, d);
+                    d = fmaf(bf16lo(uv.w), tb.z, d);
+                    d = fmaf(bf16hi(uv.w), tb.w, d);
+                }
+            }
             if (Su.has_w && row < Su.bw.nrows) {
                 const DecodeSeg &sg = p.seg[Su.bw.sp];
                 if (Su.rw > 0 && p.lag > 0)
@@ -1082,16 +1181,26 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             for (int cc = 0; cc < nch; ++cc) {
                 const uint32_t cbase = sbase + (uint32_t)cc * kDecodeChunkBytes;
                 const int kk0 = (c_lo + cc) * CK;
-                if (kk0 + CK <= K)
+                if (fused && t == 0 && t_sp >= 0) {
+                    const int t_r = p.seg[t_sp].r;
+                    const uint32_t tv_lane =
+                        smem_addr(vs) +
+                        (uint32_t)((((lane & 7) + ((lane >> 4) << 3)) * t_r + (((lane >> 3) & 1) << 3)) * 2);
+                    if (kk0 + CK <= K)
+                        w0v_chunk<NT, FTA, true>(acc, acct, cbase, swz, kk0, K, nvalid, xs_lane, tv_lane, t_r, q);
+                    else
+                        w0v_chunk<NT, FTA, false>(acc, acct, cbase, swz, kk0, K, nvalid, xs_lane, tv_lane, t_r, q);
+                } else if (kk0 + CK <= K) {
                     w0_chunk<NT, XS, true>(acc, cbase, swz, kk0, K, nvalid, xs_lane, xg_lane);
-                else
+                } else {
                     w0_chunk<NT, XS, false>(acc, cbase, swz, kk0, K, nvalid, xs_lane, xg_lane);
+                }
             }
             release_slot();
         }
 
         // ---- U part of block t - lag: U T ----
-        const bool u_part = S.has_u && S.ru > 0;
+        const bool u_part = S.has_u && S.ru > 0 && !fused;
         const DecodeSeg &sgu = p.seg[S.bu.sp];
         if (u_part && p.u_bulk && !p.u_stage && ok) {
             int u_lo, u_hi;
@@ -1165,6 +1274,17 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             }
         }
 
+        // fused T: this warp's partial sums go to the second step buffer,
+        // which step 1 fills only after T is added up
+        if (fused && t == 0 && ok) {
+            float *tred = red + (size_t)NW * 32 * 8 * NT;
+#pragma unroll
+            for (int jt = 0; jt < FTA; ++jt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<float4 *>(tred + ((size_t)(warp * FTA + jt) * NT + nt) * 128 + lane * 4) =
+                        make_float4(acct[jt][nt][0], acct[jt][nt][1], acct[jt][nt][2], acct[jt][nt][3]);
+        }
         // ---- publish this warp's sums of step t ----
         const int rbuf = t & 1;
         float *rb = red + (size_t)rbuf * NW * 32 * 8 * NT;
@@ -1187,7 +1307,7 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
         // phases need every warp), end with a CTA barrier and their epilogue;
         // elsewhere no warp waits for the others except through the two
         // buffers, and the epilogue runs one step behind.
-        const bool sync_step = SMALL || (p.t_mode == kTGrid && t <= p.lag);
+        const bool sync_step = SMALL || (p.t_mode == kTGrid && t <= p.lag) || (fused && t == 0);
         if (sync_step) {
             if (__syncthreads_or(!ok || *abort_flag != 0)) {
                 ok = false;  // every warp leaves together
@@ -1195,6 +1315,23 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
             }
         } else if (!ok) {
             break;
+        }
+        if (fused && t == 0) {
+            // T of the CTA's projection: the eight warps' partial sums, added
+            // in warp order (fragment element (j, token m) of tile jt, nt)
+            if (t_sp >= 0) {
+                const float *tred = red + (size_t)NW * 32 * 8 * NT;
+                const int t_off = p.seg[t_sp].t_off, t_r = p.seg[t_sp].r;
+                for (int i = tid; i < M * t_r; i += NTH) {
+                    const int m = i / t_r, j = i - m * t_r;
+                    const int jt = j >> 4, jr = j & 15, nt = m >> 3, col = m & 7;
+                    const int fl = (jr & 7) * 4 + (col >> 1), fe = (jr >> 3) * 2 + (col & 1);
+                    float sum = 0.f;
+                    for (int w = 0; w < NW; ++w) sum += tred[((size_t)(w * FTA + jt) * NT + nt) * 128 + fl * 4 + fe];
+                    Ts[(size_t)m * p.t_ld + t_off + j] = sum;
+                }
+            }
+            __syncthreads();
         }
         const Step cur = S;
         const float cur_sc_w = sc_w, cur_sc_u = sc_u;
@@ -1314,144 +1451,192 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
 
     // T mode.  Local when the V rows any one CTA needs stay small, with the
     // CTAs first shared out among the projections (then a CTA needs one V).
+    // Fused local T (rank <= 32, V and U staged, one projection with a delta
+    // per CTA) reads V in the W0 MMAs' shadow, so when a CTA has at most two
+    // blocks it takes a larger V rather than the grid-wide exchange.
     p.a.seg_split = 0;
     p.a.t_mode = kTNone;
+    p.a.t_fused = 0;
+    bool fusable = any_r && v_ok && p.a.u_bulk && max_r <= kDecodeFusedMaxRank && p.a.M <= 8;
+    size_t worst = 0;
     if (any_r) {
         if (blocks > grid && p.a.nseg > 1) {
             split_ctas(p.a, grid);
             p.a.seg_split = 1;
         }
         p.a.t_mode = kTLocal;
-        size_t worst = 0;
+        int most = 0;
         for (int c = 0; c < grid; ++c) {
             int lo, hi;
             cta_blocks(p.a, c, grid, lo, hi);
             size_t bytes = 0;
+            int touched = 0;
             for (int i = 0; i < p.a.nseg; ++i)
-                if (seg_touched(p.a.seg[i], lo, hi)) bytes += (size_t)p.a.K * p.a.seg[i].r * 2;
+                if (seg_touched(p.a.seg[i], lo, hi)) {
+                    bytes += (size_t)p.a.K * p.a.seg[i].r * 2;
+                    ++touched;
+                }
             worst = bytes > worst ? bytes : worst;
+            most = hi - lo > most ? hi - lo : most;
+            if (touched > 1) fusable = false;
         }
-        if (worst > kLocalVBytes) {
+        const size_t local_max = (fusable && most <= 2) ? kFusedLocalVBytes : kLocalVBytes;
+        if (worst > local_max) {
             p.a.t_mode = kTGrid;
             p.a.seg_split = 0;
+            fusable = false;
         }
     }
-    int min_blocks = blocks, max_blocks = 0;
-    size_t v_bytes = 0, u_bytes = 0;
-    for (int c = 0; c < grid; ++c) {
-        int lo, hi;
-        cta_blocks(p.a, c, grid, lo, hi);
-        min_blocks = hi - lo < min_blocks ? hi - lo : min_blocks;
-        max_blocks = hi - lo > max_blocks ? hi - lo : max_blocks;
-        size_t bytes = 0;
-        for (int i = 0; i < p.a.nseg; ++i) {
-            int k0, k1;
-            v_range(p.a, i, c, grid, lo, hi, k0, k1);
-            bytes += (size_t)(k1 - k0) * p.a.seg[i].r * 2;
-        }
-        v_bytes = bytes > v_bytes ? bytes : v_bytes;
-        size_t ub = 0;
-        for (int i = 0; i < p.a.nseg; ++i) {
-            if (p.a.seg[i].r == 0) continue;
-            int b0, b1;
-            seg_block_range(p.a.seg[i], lo, hi, b0, b1);
-            ub += (size_t)(b1 - b0) * BR * p.a.seg[i].r * 2;
-        }
-        u_bytes = ub > u_bytes ? ub : u_bytes;
-    }
-    // grid mode: partial sums in step 1, the reduction in step 2, T loaded in
-    // step 3, where the U part of block 0 runs
-    p.a.lag = p.a.t_mode == kTGrid ? kDecodeMaxLag : 0;
-    p.a.x_ld = p.a.K + 8;
 
-    // Shared memory: the compact variant (two CTAs per SM) for calls whose
-    // per-CTA stream is short, when x fits beside a one-slot ring; otherwise
-    // the full-size one.  Within the budget: x, then the staged V rows, then
-    // more ring slots (up to 192 KB of ring).
-    const size_t cta_bytes = (size_t)max_blocks * BR * ((size_t)p.a.K + (size_t)max_r) * 2;
     bool done = false;
-    for (int pass = 0; pass < 2 && !done; ++pass) {
-        const bool small = pass == 0;
-        if (small && cta_bytes > kSmallCtaBytes) continue;
-        const uint32_t budget = small ? kSmallSmem : kDecodeMaxSmem;
-        p.a.slots = 1;
-        p.a.x_smem = 1;
-        p.a.v_stage = 0;
-        p.a.v_bytes = 0;
-        p.a.v_in_ring = 0;
-        p.a.u_stage = 0;
-        p.a.u_bytes = 0;
-        if (smem_layout(p.a, NT).total > budget) {
-            if (small) continue;
-            p.a.x_smem = 0;
+    for (int attempt = 0; !done; ++attempt) {
+        if (attempt > 0) {
+            // a local-mode V that no layout stages: the grid-wide exchange instead
+            if (attempt > 1 || p.a.t_mode != kTLocal || worst <= kLocalVBytes) return WL_ERR_UNSUPPORTED;
+            p.a.t_mode = kTGrid;
+            p.a.seg_split = 0;
+            fusable = false;
         }
-        // Most ring slots that fit the budget with the current choices.
-        auto grow_slots = [&]() {
-            p.a.slots = 1;
-            while (p.a.slots < kDecodeMaxSlots) {
-                ++p.a.slots;
-                const SmemLayout Lg = smem_layout(p.a, NT);
-                if (Lg.total > budget || Lg.ring_bytes > kMaxRingBytes) {
-                    --p.a.slots;
-                    break;
-                }
+        int max_blocks = 0;
+        size_t v_bytes = 0, u_bytes = 0;
+        for (int c = 0; c < grid; ++c) {
+            int lo, hi;
+            cta_blocks(p.a, c, grid, lo, hi);
+            max_blocks = hi - lo > max_blocks ? hi - lo : max_blocks;
+            size_t bytes = 0;
+            for (int i = 0; i < p.a.nseg; ++i) {
+                int k0, k1;
+                v_range(p.a, i, c, grid, lo, hi, k0, k1);
+                bytes += (size_t)(k1 - k0) * p.a.seg[i].r * 2;
             }
-        };
-        if (v_ok && v_bytes > 0) {
-            // the staged rows plus, for a ragged K, room for the rows past the
-            // last one that a 16-row k-step reads (and masks)
-            const size_t vb = v_bytes + (p.a.K % 16 ? 16 * (size_t)max_r * 2 : 0);
-            p.a.v_stage = 1;
-            p.a.v_bytes = (int)vb;
+            v_bytes = bytes > v_bytes ? bytes : v_bytes;
+            size_t ub = 0;
+            for (int i = 0; i < p.a.nseg; ++i) {
+                if (p.a.seg[i].r == 0) continue;
+                int b0, b1;
+                seg_block_range(p.a.seg[i], lo, hi, b0, b1);
+                ub += (size_t)(b1 - b0) * BR * p.a.seg[i].r * 2;
+            }
+            u_bytes = ub > u_bytes ? ub : u_bytes;
+        }
+        // the staged rows plus, for a ragged K, room for the rows past the
+        // last one that a 16-row k-step reads (and masks)
+        const size_t vb = v_bytes + (p.a.K % 16 ? 16 * (size_t)max_r * 2 : 0);
+        // grid mode: partial sums in step 1, the reduction in step 2, T loaded in
+        // step 3, where the U part of block 0 runs
+        p.a.lag = p.a.t_mode == kTGrid ? kDecodeMaxLag : 0;
+        p.a.x_ld = p.a.K + 8;
+
+        // Shared memory: the compact variant (two CTAs per SM) for calls whose
+        // per-CTA stream is short, when x fits beside a one-slot ring; otherwise
+        // the full-size one.  Within the budget: x, then the staged V rows, then
+        // more ring slots (up to 192 KB of ring).
+        const size_t cta_bytes = (size_t)max_blocks * BR * ((size_t)p.a.K + (size_t)max_r) * 2;
+        for (int pass = 0; pass < 2 && !done; ++pass) {
+            const bool small = pass == 0;
+            if (small && cta_bytes > kSmallCtaBytes) continue;
+            const uint32_t budget = small ? kSmallSmem : kDecodeMaxSmem;
+            p.a.slots = 1;
+            p.a.x_smem = 1;
+            p.a.v_stage = 0;
+            p.a.v_bytes = 0;
             p.a.v_in_ring = 0;
-            int own_slots = 0;
-            if (smem_layout(p.a, NT).total <= budget) {
-                grow_slots();
-                own_slots = p.a.slots;
-            }
-            // or in the ring's last slot level, when that holds them and
-            // leaves more slots for the stream
-            p.a.v_in_ring = 1;
-            grow_slots();
-            const uint32_t level = (uint32_t)NW * p.a.slot_chunks * kDecodeChunkBytes;
-            const bool ring_ok = p.a.slots >= 2 && vb <= level && smem_layout(p.a, NT).total <= budget;
-            if (!(ring_ok && p.a.slots > own_slots)) {
-                p.a.v_in_ring = 0;
-                if (own_slots > 0) {
-                    p.a.slots = own_slots;
-                } else {
-                    p.a.v_stage = 0;
-                    p.a.v_bytes = 0;
-                }
-            }
-        }
-        if (!p.a.v_stage) grow_slots();
-        if (small && p.a.u_bulk && u_bytes > 0 && !p.a.v_in_ring) {
-            // the compact variant's ring is shallow: U rides outside it
-            const int slots = p.a.slots;
-            p.a.u_stage = 1;
-            p.a.u_bytes = (int)u_bytes;
-            p.a.slots = 1;
+            p.a.u_stage = 0;
+            p.a.u_bytes = 0;
+            p.a.t_fused = 0;
             if (smem_layout(p.a, NT).total > budget) {
+                if (small) continue;
+                p.a.x_smem = 0;
+            }
+            // Most ring slots that fit the budget with the current choices.
+            auto grow_slots = [&]() {
+                p.a.slots = 1;
+                while (p.a.slots < kDecodeMaxSlots) {
+                    ++p.a.slots;
+                    const SmemLayout Lg = smem_layout(p.a, NT);
+                    if (Lg.total > budget || Lg.ring_bytes > kMaxRingBytes) {
+                        --p.a.slots;
+                        break;
+                    }
+                }
+            };
+            if (fusable && v_bytes > 0 && p.a.x_smem) {
+                // fused local T: V and U rows in their own regions
+                p.a.t_fused = 1;
+                p.a.v_stage = 1;
+                p.a.v_bytes = (int)vb;
+                p.a.u_stage = 1;
+                p.a.u_bytes = (int)u_bytes;
+                if (smem_layout(p.a, NT).total <= budget) {
+                    grow_slots();
+                    plan->small = small ? 1 : 0;
+                    done = true;
+                    continue;
+                }
+                p.a.t_fused = 0;
+                p.a.v_stage = 0;
+                p.a.v_bytes = 0;
                 p.a.u_stage = 0;
                 p.a.u_bytes = 0;
-                p.a.slots = slots;
-            } else {
-                grow_slots();
             }
+            if (v_ok && v_bytes > 0) {
+                p.a.v_stage = 1;
+                p.a.v_bytes = (int)vb;
+                p.a.v_in_ring = 0;
+                int own_slots = 0;
+                if (smem_layout(p.a, NT).total <= budget) {
+                    grow_slots();
+                    own_slots = p.a.slots;
+                }
+                // or in the ring's last slot level, when that holds them and
+                // leaves more slots for the stream
+                p.a.v_in_ring = 1;
+                grow_slots();
+                const uint32_t level = (uint32_t)NW * p.a.slot_chunks * kDecodeChunkBytes;
+                const bool ring_ok = p.a.slots >= 2 && vb <= level && smem_layout(p.a, NT).total <= budget;
+                if (!(ring_ok && p.a.slots > own_slots)) {
+                    p.a.v_in_ring = 0;
+                    if (own_slots > 0) {
+                        p.a.slots = own_slots;
+                    } else {
+                        p.a.v_stage = 0;
+                        p.a.v_bytes = 0;
+                    }
+                }
+            }
+            // The compact variant only with V staged: without it T is formed
+            // element by element on the CUDA cores, far slower than the
+            // full-size variant's staged rows.
+            if (small && v_ok && v_bytes > 0 && !p.a.v_stage) continue;
+            if (!p.a.v_stage) grow_slots();
+            if (small && p.a.u_bulk && u_bytes > 0 && !p.a.v_in_ring) {
+                // the compact variant's ring is shallow: U rides outside it
+                const int slots = p.a.slots;
+                p.a.u_stage = 1;
+                p.a.u_bytes = (int)u_bytes;
+                p.a.slots = 1;
+                if (smem_layout(p.a, NT).total > budget) {
+                    p.a.u_stage = 0;
+                    p.a.u_bytes = 0;
+                    p.a.slots = slots;
+                } else {
+                    grow_slots();
+                }
+            }
+            if (smem_layout(p.a, NT).total > budget) return WL_ERR_UNSUPPORTED;
+            plan->small = small ? 1 : 0;
+            done = true;
         }
-        if (smem_layout(p.a, NT).total > budget) return WL_ERR_UNSUPPORTED;
-        plan->small = small ? 1 : 0;
-        done = true;
+        // local T over a large V only with the rows staged
+        if (done && p.a.t_mode == kTLocal && worst > kLocalVBytes && !p.a.v_stage) done = false;
     }
-    if (!done) return WL_ERR_UNSUPPORTED;
     plan->grid = grid;
     plan->smem = smem_layout(p.a, NT).total;
     plan->tpart_bytes = p.a.t_mode == kTGrid ? (size_t)(grid + 1) * p.a.M * p.a.t_ld * sizeof(float) : 0;
     return WL_OK;
 }
 
-template <int NT, bool XS, bool SMALL>
+template <int NT, bool XS, bool SMALL, int FT>
 static cudaError_t launch_decode_v(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
     // Opt in to the large shared-memory carve-out once per device: both
     // variants run with all of the SM's shared memory configured, so the
@@ -1462,10 +1647,10 @@ static cudaError_t launch_decode_v(const DecodeParams &p, const DecodePlan &plan
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL, FT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kDecodeMaxSmem);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL, FT>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
@@ -1480,18 +1665,33 @@ static cudaError_t launch_decode_v(const DecodeParams &p, const DecodePlan &plan
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<NT, XS, SMALL>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<NT, XS, SMALL, FT>, p);
 }
 
 template <int NT>
 static cudaError_t launch_decode_nt(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
     if (plan.small)  // the planner takes the compact variant only with x in shared memory
-        return p.a.x_smem ? launch_decode_v<NT, true, true>(p, plan, stream) : cudaErrorInvalidValue;
-    return p.a.x_smem ? launch_decode_v<NT, true, false>(p, plan, stream)
-                    : launch_decode_v<NT, false, false>(p, plan, stream);
+        return p.a.x_smem ? launch_decode_v<NT, true, true, 0>(p, plan, stream) : cudaErrorInvalidValue;
+    return p.a.x_smem ? launch_decode_v<NT, true, false, 0>(p, plan, stream)
+                    : launch_decode_v<NT, false, false, 0>(p, plan, stream);
+}
+
+// Fused local T: M <= 8, x in shared memory, one or two 16-column tiles of the rank.
+template <int FT>
+static cudaError_t launch_decode_fused(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+    return plan.small ? launch_decode_v<1, true, true, FT>(p, plan, stream)
+                      : launch_decode_v<1, true, false, FT>(p, plan, stream);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+    if (p.a.t_fused) {
+        if (p.a.M > 8 || !p.a.x_smem) return cudaErrorInvalidValue;
+        int max_r = 0;
+        for (int i = 0; i < p.a.nseg; ++i) max_r = p.a.seg[i].r > max_r ? p.a.seg[i].r : max_r;
+        if (max_r <= 16) return launch_decode_fused<1>(p, plan, stream);
+        if (max_r <= 2 * 16) return launch_decode_fused<2>(p, plan, stream);
+        return cudaErrorInvalidValue;
+    }
     if (p.a.M <= 8) return launch_decode_nt<1>(p, plan, stream);
     if (p.a.M <= 16) return launch_decode_nt<2>(p, plan, stream);
     return cudaErrorInvalidValue;

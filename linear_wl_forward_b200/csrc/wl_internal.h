@@ -24,6 +24,7 @@ constexpr int kDecodeMaxSlotChunks = 4;   // a ring slot holds up to 16 rows x 2
 constexpr int kDecodeMaxSlots = 4;        // ring slots per warp
 constexpr int kDecodeTMaxFloats = 12288;  // M (rounded up to 8) * (sum of ranks) in shared memory
 constexpr int kDecodeMaxLag = 3;          // grid T mode: blocks by which the U part of a block trails its W0 part
+constexpr int kDecodeFusedMaxRank = 32;   // fused local T: largest rank (two 16-column tiles of T per warp)
 
 // How a CTA obtains T = V^T x.
 enum DecodeTMode : int {
@@ -70,6 +71,8 @@ struct DecodeArgs {
     int v_in_ring;    // they sit in the ring's last slot level until T's sums are formed
     int u_stage;      // each CTA bulk-copies its blocks' U rows into shared memory (not through the ring)
     int u_bytes;      // shared memory they need (largest over the CTAs)
+    int t_fused;      // kTLocal: T's MMAs run inside the first step's W0 part (sharing its x
+                      // fragments) and every epilogue adds U T from the staged U rows
     const __nv_bfloat16 *x;
     float *Tpart;     // kTGrid: [grid][M][t_ld] partial sums, then [M][t_ld] final T
     unsigned int *sync;  // kTGrid: [0], [1] arrival counts, [2] departures; self-resetting

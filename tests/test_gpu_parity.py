@@ -31,7 +31,11 @@ def test_tiny_band_both_layers(path):
 DECODE_CASES = [(1, 1, 8, 0), (1, 37, 24, 5), (2, 300, 1000, 16), (3, 513, 1032, 64),
                 (4, 257, 2056, 256), (1, 2000, 3080, 8), (4, 129, 64, 1024), (2, 64, 8, 3),
                 (8, 700, 4104, 24), (13, 333, 520, 256), (16, 2048, 5376, 256), (9, 17, 16, 7),
-                (16, 40, 8, 0), (5, 4000, 136, 1000)]
+                (16, 40, 8, 0), (5, 4000, 136, 1000),
+                # T formed inside the first step (rank <= 32, M <= 8): two-block
+                # CTAs with a ragged K, V of 128 KB (full-size variant), a rank
+                # of one and a half 16-column tiles with V above 96 KB
+                (5, 3000, 1160, 32), (1, 1152, 4096, 16), (7, 700, 2056, 24), (1, 1152, 4096, 8)]
 GEMM_CASES = [(1, 37, 24, 5), (5, 300, 200, 16), (130, 513, 1000, 64), (257, 255, 136, 72),
               (64, 1024, 520, 256), (200, 77, 64, 0), (129, 600, 2056, 4), (16, 256, 256, 1024),
               (300, 1, 8, 8)]
