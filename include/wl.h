@@ -214,6 +214,37 @@ wl_status wl_materialize_weight(const wl_bf16 *W0, const float *s, const wl_bf16
                                 const wl_bf16 *V, wl_bf16 *W_eff, int N, int K, int r,
                                 void *stream);
 
+/* What the decode kernel would do with a call: the host-side plan, made
+ * without a GPU (no tensor maps, no launch).  The pointers in `projs` are
+ * checked for NULL and alignment only, never dereferenced, so stand-in
+ * values describe a call before its buffers exist.  t_mode: 0 = no delta,
+ * 1 = local (each CTA forms its T slices from the staged V rows), 2 = grid
+ * (partial sums over K slices meet through two grid-wide counts). */
+typedef struct {
+    int auto_decode;  /* WL_PATH_AUTO takes the decode kernel for this call  */
+    int grid;         /* CTAs, at most one per SM (two for compact calls)    */
+    int compact;      /* the two-CTA/SM variant (<= 110 KB shared memory)     */
+    long long smem_bytes; /* dynamic shared memory per CTA                  */
+    int t_mode;       /* see above                                          */
+    int t_fused;      /* T formed inside the first step's W0 MMAs           */
+    int seg_split;    /* CTAs shared out among the stacked projections      */
+    int slots;        /* ring slots per warp                                */
+    int slot_chunks;  /* 64-column W0 chunks per slot                       */
+    int x_smem;       /* x staged in shared memory                          */
+    int v_stage;      /* the V rows for T staged in shared memory           */
+    int v_in_ring;    /* ... in the ring's last slot level                  */
+    int u_stage;      /* the U rows of the CTA's blocks staged              */
+    int lag;          /* grid mode: steps by which a block's U part trails  */
+} wl_decode_plan;
+
+/* Fills *out for the call (M tokens, K, P projections as wl_stacked_forward
+ * takes them) on a GPU with num_sms SMs.  out->auto_decode is set whenever
+ * the arguments are valid.  Returns WL_ERR_UNSUPPORTED for shapes the decode
+ * kernel declines (M outside 1..WL_DECODE_MAX_M, K < 8, too many T values),
+ * and the argument errors of wl_stacked_forward. */
+wl_status wl_describe_decode_plan(int M, int K, const wl_proj *projs, int P, int num_sms,
+                                  wl_decode_plan *out);
+
 /* Static description of a status code. */
 const char *wl_status_string(wl_status status);
 

@@ -12,7 +12,7 @@ import os
 
 __all__ = [
     "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
-    "materialize_weight",
+    "materialize_weight", "describe_decode_plan", "DecodePlan",
     "decompose",
     "relative_frobenius_error", "last_device_status", "wait_probe", "PATHS",
     "DECODE_MAX_M", "MAX_RANK", "MAX_PROJ", "STATUS",
@@ -42,6 +42,15 @@ class _Proj(ctypes.Structure):
                 ("r", ctypes.c_int)]
 
 
+class DecodePlan(ctypes.Structure):
+    """wl_decode_plan of include/wl.h."""
+    _fields_ = [("auto_decode", ctypes.c_int), ("grid", ctypes.c_int), ("compact", ctypes.c_int),
+                ("smem_bytes", ctypes.c_longlong), ("t_mode", ctypes.c_int), ("t_fused", ctypes.c_int),
+                ("seg_split", ctypes.c_int), ("slots", ctypes.c_int), ("slot_chunks", ctypes.c_int),
+                ("x_smem", ctypes.c_int), ("v_stage", ctypes.c_int), ("v_in_ring", ctypes.c_int),
+                ("u_stage", ctypes.c_int), ("lag", ctypes.c_int)]
+
+
 _lib = None
 
 
@@ -60,6 +69,8 @@ def lib():
         L.wl_decompose.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp]
         L.wl_decompose_als.argtypes = [vp, ci, ci, ci, ci, ci, vp, ci, vp, vp, vp, vp, vp]
         L.wl_materialize_weight.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, vp]
+        L.wl_describe_decode_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci,
+                                              ctypes.POINTER(DecodePlan)]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
         L.wl_relative_frobenius_error.restype = ctypes.c_double
         L.wl_status_string.argtypes = [ci]
@@ -68,7 +79,7 @@ def lib():
         L.wl_wait_probe.argtypes = [cll, vp]
         L.wl_version.restype = ci
         for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose", "wl_decompose_als",
-                     "wl_materialize_weight",
+                     "wl_materialize_weight", "wl_describe_decode_plan",
                      "wl_last_device_status", "wl_wait_probe"):
             getattr(L, name).restype = ci
         _lib = L
@@ -196,6 +207,26 @@ def materialize_weight(W0, s, U, V, out=None, stream=None):
         _dev_ptr(out, torch.bfloat16, "out", (N, K)), N, K, r, _stream_handle(stream)),
         "wl_materialize_weight")
     return out
+
+
+def describe_decode_plan(M: int, K: int, projs, num_sms: int = 148) -> dict:
+    """The decode kernel's host-side plan for a call, made without a GPU.
+
+    ``projs`` holds ``(N, r)`` pairs, or ``(N, r, uv_offset)`` with U and V
+    placed ``uv_offset`` bytes past a 16-byte boundary.  The pointers handed
+    to the library are stand-ins: it checks them for NULL and alignment only.
+    Raises WLError for shapes the decode kernel declines."""
+    arr = (_Proj * len(projs))()
+    for i, q in enumerate(projs):
+        N, r = q[0], q[1]
+        off = q[2] if len(q) > 2 else 0
+        base = (i + 1) << 32
+        arr[i] = _Proj(base, base + (1 << 28), (base + (2 << 28) + off) if r else None,
+                       (base + (3 << 28) + off) if r else None, base + (4 << 28), N, r)
+    out = DecodePlan()
+    _check(lib().wl_describe_decode_plan(M, K, arr, len(projs), num_sms, ctypes.byref(out)),
+           "wl_describe_decode_plan")
+    return {name: getattr(out, name) for name, _ in DecodePlan._fields_}
 
 
 def last_device_status(stream=None) -> int:

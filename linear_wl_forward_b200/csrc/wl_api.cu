@@ -540,6 +540,38 @@ wl_status wl_materialize_weight(const wl_bf16 *W0, const float *s, const wl_bf16
         static_cast<cudaStream_t>(stream)));
 }
 
+wl_status wl_describe_decode_plan(int M, int K, const wl_proj *projs, int P, int num_sms,
+                                  wl_decode_plan *out) {
+    if (!out || num_sms < 1) return WL_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof *out);
+    // x is not part of a plan: validate the projections against an aligned stand-in
+    alignas(16) static const unsigned char no_x[16] = {};
+    wl_status st = wl::validate(reinterpret_cast<const wl_bf16 *>(no_x), M, K, projs, P, WL_PATH_DECODE);
+    if (st != WL_OK) return st;
+    out->auto_decode = wl::auto_decode(M, projs, P) ? 1 : 0;
+    if (M < 1 || K < 8) return WL_ERR_UNSUPPORTED;
+    static wl::DecodeParams dp;  // large (tensor maps); guarded by g_mu
+    std::lock_guard<std::mutex> lock(wl::g_mu);
+    if (!wl::build_decode_params(nullptr, M, K, projs, P, dp)) return WL_ERR_UNSUPPORTED;
+    wl::DecodePlan plan;
+    if ((st = wl::plan_decode(dp, num_sms, &plan, false)) != WL_OK) return st;
+    const wl::DecodeArgs &a = dp.a;
+    out->grid = plan.grid;
+    out->compact = plan.small;
+    out->smem_bytes = (long long)plan.smem;
+    out->t_mode = a.t_mode;
+    out->t_fused = a.t_fused;
+    out->seg_split = a.seg_split;
+    out->slots = a.slots;
+    out->slot_chunks = a.slot_chunks;
+    out->x_smem = a.x_smem;
+    out->v_stage = a.v_stage;
+    out->v_in_ring = a.v_in_ring;
+    out->u_stage = a.u_stage;
+    out->lag = a.lag;
+    return WL_OK;
+}
+
 wl_status wl_last_device_status(void *stream) {
     std::lock_guard<std::mutex> lock(wl::g_mu);
     wl::DevicePool *pool = nullptr;

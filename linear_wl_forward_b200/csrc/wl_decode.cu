@@ -1405,7 +1405,7 @@ void split_ctas(DecodeArgs &p, int grid) {
 
 }  // namespace
 
-wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
+wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan, bool encode_maps) {
     if (p.a.M < 1 || p.a.M > WL_DECODE_MAX_M || p.a.K < 8 || p.a.nseg < 1 || num_sms < 1) return WL_ERR_UNSUPPORTED;
     const int NT = (p.a.M + 7) / 8;
     if ((size_t)8 * NT * p.a.t_ld > (size_t)kDecodeTMaxFloats) return WL_ERR_UNSUPPORTED;
@@ -1439,7 +1439,7 @@ wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan) {
     p.a.w3d = (p.a.K % CK == 0 && p.a.slot_chunks >= 2) ? 1 : 0;
 
     wl_status st;
-    for (int i = 0; i < p.a.nseg; ++i) {
+    for (int i = 0; encode_maps && i < p.a.nseg; ++i) {
         const DecodeSeg &sg = p.a.seg[i];
         if ((st = encode_map_2d(&p.tm_w[i], sg.W0, p.a.K, sg.N, p.a.K, CK, BR)) != WL_OK) return st;
         if (p.a.w3d && (st = encode_map_3d(&p.tm_w3[i], sg.W0, CK, sg.N, p.a.K / CK, (uint64_t)p.a.K * 2, CK * 2, CK,

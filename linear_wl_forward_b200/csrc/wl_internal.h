@@ -98,7 +98,9 @@ struct DecodePlan {
 // shared-memory choices; returns WL_ERR_UNSUPPORTED if the shape cannot take
 // the decode path (M above WL_DECODE_MAX_M, or M rounded up to 8 times the sum
 // of ranks above kDecodeTMaxFloats).
-wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan);
+// encode_maps = false plans without the tensor maps (host logic only: no
+// driver call, the pointers are only checked for alignment).
+wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan, bool encode_maps = true);
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
 
 // 2-D / 3-D bf16 tensor maps with 128-byte swizzling; out-of-range reads give 0.
