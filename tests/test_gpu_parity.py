@@ -193,3 +193,14 @@ def test_prepared_matches_stacked():
             for a, b in zip(ref, got):
                 assert torch.equal(a, b)
         assert wl.last_device_status() == 0
+
+
+@pytest.mark.parametrize("M,ranks", [(1, [0, 16, 32]), (2, [0, 16]), (8, [16, 0, 8])])
+def test_stacked_fused_t_with_rank_zero_projection(M, ranks):
+    """T formed inside the first step, in a stacked call where some CTAs' rows
+    have no delta (they stage no V or U rows) and the ranks need one or two
+    16-column tiles of T."""
+    plan = wl.describe_decode_plan(M, 520, [(n, r) for n, r in zip([300, 200, 40], ranks)])
+    assert plan["t_fused"] == 1
+    call = wl_inputs.random_case(60 + M, M, [300, 200, 40][:len(ranks)], 520, ranks, P=len(ranks))
+    check_call(call, "decode")
