@@ -29,6 +29,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -270,8 +271,16 @@ def traffic_from_profile(kernel, call):
     if not rec:
         return None
     src = os.path.join(ROOT, "linear_wl_forward_b200", "csrc", rec["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["dram_bytes_per_launch"] if h == rec["source_sha"] else None
+    return rec["dram_bytes_per_launch"] if kernel_source_sha(src) == rec["source_sha"] else None
+
+
+def kernel_source_sha(path):
+    """Hash of a CUDA source with its comments and whitespace removed: the
+    code the counters were taken on (a comment edit does not void them)."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()[:16]
 
 
 # -------------------------------------------------------------- secondary --

@@ -34,9 +34,14 @@
 // T = V^T x is formed inside the same kernel ("cooperative vtx" of the pages'
 // custom op), one of two ways chosen per call on the host:
 //  * local: when each CTA's V is small, the CTA reads all of it (bulk-copied
-//    into shared memory before the wait when it fits) and forms its T slices
-//    before the first block: warp MMAs with A = V^T read by ldmatrix.trans,
-//    the warps splitting the k-steps (CUDA cores when V cannot be staged);
+//    into shared memory before the wait when it fits).  Fused (M <= 8, rank
+//    <= 32, one projection with a delta per CTA; a variant of its own): the
+//    V^T x MMAs run inside the first step's W0 loop on the same x fragments,
+//    each warp over its own K chunks, the eight partial sums are added after
+//    that step's barrier, and every epilogue adds U T on the CUDA cores from
+//    the staged U rows.  Otherwise the CTA forms its T slices before the
+//    first block: warp MMAs with A = V^T read by ldmatrix.trans, the warps
+//    splitting the k-steps (CUDA cores when V cannot be staged);
 //  * grid: otherwise each CTA forms partial sums over a 1/grid slice of K for
 //    every projection (the warps splitting the 16-column tiles of r) and
 //    writes them to scratch (phase A); then it waits for all CTAs' partials
