@@ -370,6 +370,10 @@ __device__ __forceinline__ void w0_chunk(float (&acc)[NT][4], uint32_t cbase, co
 // w0_chunk plus, on the same x fragments, the chunk's share of T = V^T x for
 // the rank r <= 32 of the CTA's projection (fused local T): A = V^T from the
 // staged V rows (row k at k * r) through ldmatrix.trans, rows past K masked.
+// A tile's columns past r (FT = 2 with r <= 24, or a projection of rank 16
+// in a call whose largest rank needs two tiles) read the following rows'
+// values, at most 32 bytes past the staged rows and still inside the CTA's
+// shared memory; their sums land in T columns that nothing reads.
 template <int NT, int FT, bool FULL>
 __device__ __forceinline__ void w0v_chunk(float (&acc)[NT][4], float (&acct)[FT][NT][4], uint32_t cbase,
                                           const uint32_t (&swz)[CK / 16], int kk0, int K,
