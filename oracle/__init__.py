@@ -8,6 +8,8 @@ code with the CUDA library (``linear_wl_forward_b200``) and never imports it.
   factored and dense-W_eff forms.
 * ``decompose`` / ``relative_frobenius_error``: numpy fp64 decomposition
   (``decompose.py``).
+* ``nvfp4``: the NVFP4 weight encoding (E2M1 codes, E4M3 block scales, an
+  fp32 tensor scale) and the forward over an NVFP4-encoded W0 (``nvfp4.py``).
 """
 from __future__ import annotations
 

@@ -144,3 +144,67 @@ def test_decompose_planted_mistake_is_caught(monkeypatch, name):
     head, tail = text[:cut], text[cut:]
     assert head.count(old) == 1, f"mutation site of {name} not found exactly once"
     assert _dfailures(monkeypatch, head.replace(old, new) + tail) > 0, f"no pin catches the mutant {name}"
+
+
+# ----------------------------------------------------------------- NVFP4 ---
+# The NVFP4 pins (test_oracle_nvfp4) must catch a plausible mistake in the
+# encoding oracle: wrong nibble order, exponent bias or subnormal step, ties
+# away from zero, a dropped sign, a mis-scaled block or tensor scale, or a
+# forward that drops a term.
+import test_oracle_nvfp4 as npins  # noqa: E402
+
+NSRC = os.path.join(os.path.dirname(oracle.__file__), "nvfp4.py")
+
+NMUTANTS = {
+    "nibble_order": ("return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)",
+                     "return (c[:, 1::2] | (c[:, 0::2] << 4)).astype(np.uint8)"),
+    "e4m3_bias": ("np.exp2(e - 7.0)", "np.exp2(e - 8.0)"),
+    "e4m3_subnormal_step": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
+    "e2m1_subnormal_step": ("(c & 1) * 0.5 if (c >> 1) == 0", "(c & 1) * 0.25 if (c >> 1) == 0"),
+    "ties_away_from_zero": ("pick_hi = (dhi < dlo) | ((dhi == dlo) & even[hi])", "pick_hi = dhi <= dlo"),
+    "sign_dropped": ("return (idx + np.where(np.signbit(v), 8, 0)).astype(np.uint8)",
+                     "return idx.astype(np.uint8)"),
+    "block_scale_over_4": ("sbytes = e4m3_encode(bmax / (E2M1_MAX * tensor_scale))",
+                           "sbytes = e4m3_encode(bmax / (4.0 * tensor_scale))"),
+    "tensor_scale_without_6": ("tensor_scale = amax / (E2M1_MAX * E4M3_MAX)", "tensor_scale = amax / E4M3_MAX"),
+    "dequant_drops_tensor_scale": ("return (vals * e4m3_decode(sbytes)[:, :, None] * tensor_scale).reshape(N, K)",
+                                   "return (vals * e4m3_decode(sbytes)[:, :, None]).reshape(N, K)"),
+    "forward_drops_scale": ("y = f64(s)[None, :] * (X @ W0.T)", "y = X @ W0.T"),
+    "forward_drops_delta": ("y = y + (X @ Vf) @ Uf.T", "y = y"),
+}
+
+
+def _npin_calls():
+    calls = [npins.test_e4m3_decode_matches_torch, npins.test_e4m3_encode_matches_torch_rounding,
+             npins.test_e2m1_rounding_brute_force, npins.test_e2m1_table_shape, npins.test_golden_blocks,
+             npins.test_lossless_round_trip, npins.test_bytes_per_element,
+             npins.test_forward_matches_the_c_oracle_on_an_exact_weight]
+    for std in (0.02, 1.0, 300.0):
+        calls.append(lambda sd=std: npins.test_rounding_error_bound(sd))
+    return calls
+
+
+def _nfailures(monkeypatch, text):
+    mod = types.ModuleType("nvfp4_mutant")
+    exec(compile(text, "nvfp4_mutant.py", "exec"), mod.__dict__)
+    monkeypatch.setattr(npins, "nvfp4", mod)
+    failed = 0
+    for call in _npin_calls():
+        try:
+            call()
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    monkeypatch.undo()
+    return failed
+
+
+def test_nvfp4_unmodified_passes_every_pin(monkeypatch):
+    assert _nfailures(monkeypatch, open(NSRC).read()) == 0
+
+
+@pytest.mark.parametrize("name", sorted(NMUTANTS))
+def test_nvfp4_planted_mistake_is_caught(monkeypatch, name):
+    old, new = NMUTANTS[name]
+    text = open(NSRC).read()
+    assert text.count(old) == 1, f"mutation site of {name} not found exactly once"
+    assert _nfailures(monkeypatch, text.replace(old, new)) > 0, f"no pin catches the mutant {name}"
