@@ -214,6 +214,29 @@ wl_status wl_materialize_weight(const wl_bf16 *W0, const float *s, const wl_bf16
                                 const wl_bf16 *V, wl_bf16 *W_eff, int N, int K, int r,
                                 void *stream);
 
+/* NVFP4 encoding of a weight for 4-bit weight streaming ("Compression",
+ * section "NVFP4: 3.18x smaller weights": packed 4-bit weights plus one
+ * float8_e4m3fn block scale per 16 elements, 0.5625 bytes per element,
+ * quantised at load time).  Host memory, synchronous:
+ *   W      : N x K fp32, row-major, finite
+ *   codes  : N x K/2 bytes (written): FP4 E2M1 codes, element 2i in the low
+ *            nibble of byte i, 2i + 1 in the high nibble
+ *   scales : N x K/16 bytes (written): FP8 E4M3 scale of each 16-element
+ *            block along K
+ *   tensor_scale : > 0 to use as given; 0 to take max|W| / (6 * 448) rounded
+ *            to fp32 (1 for an all-zero W); the value used is written to
+ *            *tensor_scale_out
+ * Dequantised element: e2m1(code) * e4m3(scale) * tensor scale.  Block
+ * scale = max|w| of the block / (6 * tensor scale) and code = w / (block
+ * scale * tensor scale), both in fp64, rounded to nearest-even and saturated
+ * (448, 6); a block whose scale rounds to zero gets zero codes.
+ * Returns WL_ERR_ALIGNMENT unless K % 16 == 0, WL_ERR_INVALID_ARG for
+ * negative sizes, null buffers, a negative or infinite tensor_scale or a
+ * non-finite W, WL_ERR_UNSUPPORTED if the host's floating-point rounding
+ * mode is not round-to-nearest. */
+wl_status wl_quantize_nvfp4(const float *W, int N, int K, float tensor_scale, uint8_t *codes,
+                            uint8_t *scales, float *tensor_scale_out);
+
 /* What the decode kernel would do with a call: the host-side plan, made
  * without a GPU (no tensor maps, no launch).  The pointers in `projs` are
  * checked for NULL and alignment only, never dereferenced, so stand-in

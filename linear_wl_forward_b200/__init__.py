@@ -12,7 +12,7 @@ import os
 
 __all__ = [
     "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
-    "materialize_weight", "describe_decode_plan", "DecodePlan",
+    "materialize_weight", "describe_decode_plan", "DecodePlan", "quantize_nvfp4",
     "decompose",
     "relative_frobenius_error", "last_device_status", "wait_probe", "PATHS",
     "DECODE_MAX_M", "MAX_RANK", "MAX_PROJ", "STATUS",
@@ -71,6 +71,7 @@ def lib():
         L.wl_materialize_weight.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, vp]
         L.wl_describe_decode_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci,
                                               ctypes.POINTER(DecodePlan)]
+        L.wl_quantize_nvfp4.argtypes = [vp, ci, ci, ctypes.c_float, vp, vp, ctypes.POINTER(ctypes.c_float)]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
         L.wl_relative_frobenius_error.restype = ctypes.c_double
         L.wl_status_string.argtypes = [ci]
@@ -79,7 +80,7 @@ def lib():
         L.wl_wait_probe.argtypes = [cll, vp]
         L.wl_version.restype = ci
         for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose", "wl_decompose_als",
-                     "wl_materialize_weight", "wl_describe_decode_plan",
+                     "wl_materialize_weight", "wl_describe_decode_plan", "wl_quantize_nvfp4",
                      "wl_last_device_status", "wl_wait_probe"):
             getattr(L, name).restype = ci
         _lib = L
@@ -207,6 +208,22 @@ def materialize_weight(W0, s, U, V, out=None, stream=None):
         _dev_ptr(out, torch.bfloat16, "out", (N, K)), N, K, r, _stream_handle(stream)),
         "wl_materialize_weight")
     return out
+
+
+def quantize_nvfp4(W, tensor_scale: float = 0.0):
+    """NVFP4 encoding on the host (include/wl.h, wl_quantize_nvfp4).  W: N x K
+    float32 numpy array, K % 16 == 0.  Returns (codes N x K/2 uint8, scales
+    N x K/16 uint8, tensor scale); tensor_scale 0 derives it from max|W|."""
+    import numpy as np
+
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    codes = np.empty((N, K // 2), np.uint8)
+    scales = np.empty((N, max(K // 16, 0)), np.uint8)
+    ts = ctypes.c_float(0.0)
+    _check(lib().wl_quantize_nvfp4(W.ctypes.data, N, K, float(tensor_scale), codes.ctypes.data,
+                                   scales.ctypes.data, ctypes.byref(ts)), "wl_quantize_nvfp4")
+    return codes, scales, ts.value
 
 
 def describe_decode_plan(M: int, K: int, projs, num_sms: int = 148) -> dict:

@@ -19,11 +19,12 @@ per element.  What the page leaves open is read as follows:
 * storage: codes row-major, two per byte, element 2i in the low nibble and
   2i + 1 in the high nibble (N x K/2 bytes); scales row-major (N x K/16);
 * quantisation (the page says the weights are quantised at load time but not
-  how): tensor scale = max|W| / (6 * 448); block scale = the block's max|w| /
-  (6 * tensor scale), rounded to nearest-even E4M3 and saturated at 448;
-  code = w / (block scale * tensor scale) rounded to nearest-even E2M1 and
-  saturated at +-6; a block whose scale rounds to 0 gets codes 0.  These
-  divisions are taken in fp64.
+  how): tensor scale = max|W| / (6 * 448) rounded to fp32 (the stored
+  number, which the block scales are then taken against); block scale = the
+  block's max|w| / (6 * tensor scale), rounded to nearest-even E4M3 and
+  saturated at 448; code = w / (block scale * tensor scale) rounded to
+  nearest-even E2M1 and saturated at +-6; a block whose scale rounds to 0
+  gets codes 0.  These divisions are taken in fp64.
 
 Dequantised weight: w = e2m1(code) * e4m3(scale byte) * tensor scale.
 """
@@ -107,7 +108,8 @@ def quantize(W, tensor_scale=None):
     assert K % BLOCK == 0, "K must be a multiple of 16"
     if tensor_scale is None:
         amax = float(np.max(np.abs(W))) if W.size else 0.0
-        tensor_scale = amax / (E2M1_MAX * E4M3_MAX) if amax > 0 else 1.0
+        ts32 = float(np.float32(amax / (E2M1_MAX * E4M3_MAX)))
+        tensor_scale = ts32 if ts32 > 0 else 1.0  # an all-zero (or vanishing) weight
     blocks = W.reshape(N, K // BLOCK, BLOCK)
     bmax = np.max(np.abs(blocks), axis=2)
     sbytes = e4m3_encode(bmax / (E2M1_MAX * tensor_scale))

@@ -166,7 +166,7 @@ NMUTANTS = {
                      "return idx.astype(np.uint8)"),
     "block_scale_over_4": ("sbytes = e4m3_encode(bmax / (E2M1_MAX * tensor_scale))",
                            "sbytes = e4m3_encode(bmax / (4.0 * tensor_scale))"),
-    "tensor_scale_without_6": ("tensor_scale = amax / (E2M1_MAX * E4M3_MAX)", "tensor_scale = amax / E4M3_MAX"),
+    "tensor_scale_without_6": ("np.float32(amax / (E2M1_MAX * E4M3_MAX))", "np.float32(amax / E4M3_MAX)"),
     "dequant_drops_tensor_scale": ("return (vals * e4m3_decode(sbytes)[:, :, None] * tensor_scale).reshape(N, K)",
                                    "return (vals * e4m3_decode(sbytes)[:, :, None]).reshape(N, K)"),
     "forward_drops_scale": ("y = f64(s)[None, :] * (X @ W0.T)", "y = X @ W0.T"),
