@@ -82,3 +82,16 @@ def test_argument_errors():
     bad[1, 2] = np.nan
     with pytest.raises(wl.WLError):
         wl.quantize_nvfp4(bad)
+
+
+def test_seeded_nvfp4_draw_is_a_valid_encoding():
+    """The NVFP4 W0 draw (random code and scale bytes) is deterministic per
+    key and dequantises to finite weights of the bf16 draw's scale."""
+    import wl_inputs
+
+    c, s, t = wl_inputs.draw_w0_nvfp4("gemma3_1b", 1, 0, "all", "gate", 64, 1152)
+    c2, s2, t2 = wl_inputs.draw_w0_nvfp4("gemma3_1b", 1, 0, "all", "gate", 64, 1152)
+    assert (c == c2).all() and (s == s2).all() and t == t2
+    assert c.shape == (64, 576) and s.shape == (64, 72)
+    W = nvfp4.dequantize(c.numpy(), s.numpy(), t)
+    assert np.all(np.isfinite(W)) and 0.005 < W.std() < 0.05

@@ -121,6 +121,28 @@ def draw_delta(workload: str, seed: int, layer: int, family: str, N: int, K: int
     return s, U, V
 
 
+# NVFP4-encoded W0, drawn directly as bytes (no encoding arithmetic here): the
+# magnitude code of each element follows roughly the mix a block-scaled
+# Gaussian row gives (most elements small, few at the block maximum), the sign
+# is even, and the block scale bytes are E4M3 codes 0x30..0x4F (0.5 .. 15),
+# around a tensor scale of 2^-9, so dequantised weights are of order 0.01.
+NVFP4_MAG_WEIGHTS = (0.10, 0.18, 0.17, 0.14, 0.17, 0.12, 0.08, 0.04)
+NVFP4_TENSOR_SCALE = 2.0 ** -9
+
+
+def draw_w0_nvfp4(workload: str, seed: int, band: int, layer_type: str, family: str, N: int, K: int):
+    """(codes uint8[N, K/2], scale bytes uint8[N, K/16], tensor scale) of an
+    NVFP4 W0; element 2i of a row in the low nibble of byte i."""
+    assert K % 16 == 0
+    g = _gen(workload, seed, "W0nvfp4", band, layer_type, family)
+    mag = torch.multinomial(torch.tensor(NVFP4_MAG_WEIGHTS), N * K, replacement=True, generator=g)
+    sign = torch.randint(0, 2, (N * K,), generator=g)
+    nib = (mag + 8 * sign).to(torch.uint8).reshape(N, K)
+    codes = nib[:, 0::2] | (nib[:, 1::2] << 4)
+    scales = torch.randint(0x30, 0x50, (N, K // 16), generator=g).to(torch.uint8)
+    return codes.contiguous(), scales, NVFP4_TENSOR_SCALE
+
+
 def draw_x(workload: str, seed: int, M: int, K: int, tag="x") -> torch.Tensor:
     return normal_bf16((M, K), 1.0, workload, seed, tag, M, K)
 
