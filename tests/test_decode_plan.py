@@ -151,3 +151,34 @@ def test_plan_invariants_over_shapes():
         accepted += 1
         _check_invariants(M, K, projs, sms, p)
     assert accepted > 500
+
+
+def _workload_calls():
+    import wl_inputs
+
+    for stack in wl_inputs.GEMMA3_1B_STACKS:
+        fam = wl_inputs.GEMMA3_1B_FAMILIES
+        yield "gemma3", fam[stack[0]][1], [fam[f][0] for f in stack]
+    for lt in ("sliding", "full"):
+        fam = wl_inputs.gemma4_families(lt)
+        for stack in wl_inputs.gemma4_stacks(lt):
+            yield f"gemma4_{lt}", fam[stack[0]][1], [fam[f][0] for f in stack]
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 9, 16])
+@pytest.mark.parametrize("r", [16, 64, 256])
+def test_every_workload_call_plans_for_decode(M, r):
+    """Every projection stack of the Gemma-3-1B and Gemma-4-31B layers, at
+    1-16 tokens and ranks 16-256, is a shape the decode kernel takes (so
+    WL_PATH_AUTO never falls back for these), within its invariants."""
+    for name, K, Ns in _workload_calls():
+        projs = [(N, r) for N in Ns]
+        p = plan(M, K, projs)
+        _check_invariants(M, K, projs, 148, p)
+        if name == "gemma3" and M <= 8 and r <= 32:
+            # fused local T, except the down projection (K = 4096) beyond two
+            # tokens: its staged x (33-66 KB) no longer fits beside the
+            # 128 KB of V rows and a ring level, so it takes grid mode
+            fused = K < 4096 or M <= 2
+            assert p["t_fused"] == (1 if fused else 0), (name, K, Ns)
+            assert p["t_mode"] == (1 if fused else 2), (name, K, Ns)
