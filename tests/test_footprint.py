@@ -35,3 +35,36 @@ def test_call_bytes_and_flops():
     assert wb == 2 * (N * K + (N + K) * r) + 4 * N
     assert abs(wb / 1e6 - 245.0) < 0.5
     assert footprint.call_flops(4096, N, K, r) == 2 * 4096 * N * K + 2 * 4096 * K * r + 2 * 4096 * N * r
+
+
+def _gemma4_projections():
+    import wl_inputs
+
+    out = []
+    for layer in range(wl_inputs.GEMMA4_31B_LAYERS):
+        fam = wl_inputs.gemma4_families(wl_inputs.gemma4_layer_type(layer))
+        out.extend(fam.values())
+    return out
+
+
+def test_gemma4_projection_count():
+    """60 layers x (q, k, v, o, gate, up, down), with no v projection on the
+    10 full-attention layers (k = v): the page's 410 projections."""
+    assert len(_gemma4_projections()) == GOLDEN["gemma4_31b_projection_count"]["value"]
+
+
+def test_gemma4_nvfp4_bytes_match_the_page():
+    """The page's bf16 total (61.4 GB, rounded) fixes the bytes outside the
+    projections (embeddings, norms: bf16 on both sides); with the workload's
+    projection shapes at 0.5625 B per element the NVFP4 total must then
+    contain the page's 19.295 GB.  Extra projections (a v on full layers) or
+    another per-element cost (0.5 B) fall outside."""
+    g = GOLDEN["gemma4_31b_weight_bytes_GB"]
+    params = sum(N * K for N, K in _gemma4_projections())
+    lo_rest = (g["bf16"] - g["bf16_rounding"]) * 1e9 - 2 * params
+    hi_rest = (g["bf16"] + g["bf16_rounding"]) * 1e9 - 2 * params
+    assert lo_rest > 0
+    nv_lo = 0.5625 * params + lo_rest
+    nv_hi = 0.5625 * params + hi_rest
+    assert nv_lo <= (g["nvfp4"] + g["nvfp4_rounding"]) * 1e9
+    assert nv_hi >= (g["nvfp4"] - g["nvfp4_rounding"]) * 1e9
