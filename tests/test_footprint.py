@@ -68,3 +68,21 @@ def test_gemma4_nvfp4_bytes_match_the_page():
     nv_hi = 0.5625 * params + hi_rest
     assert nv_lo <= (g["nvfp4"] + g["nvfp4_rounding"]) * 1e9
     assert nv_hi >= (g["nvfp4"] - g["nvfp4_rounding"]) * 1e9
+
+
+def test_w0_is_nearly_half_of_the_g1_rank32_bundle():
+    """G = 1, rank 32, fp32 at the Gemma-3-1B dimensions: W0 (one per family)
+    is nearly half the bundle and s is negligible; W0 does not grow with the
+    rank.  Counting W0 per layer, or U and V per band, breaks the share."""
+    from linear_wl_forward_b200 import footprint
+    import wl_inputs
+
+    fam = wl_inputs.GEMMA3_1B_FAMILIES
+    L = wl_inputs.GEMMA3_1B_LAYERS
+    total = footprint.theta_bytes(fam, L, 1, 32)
+    w0 = footprint.theta_bytes(fam, 1, 1, 0) - 4 * sum(N for N, _ in fam.values())
+    s_bytes = 4 * L * sum(N for N, _ in fam.values())
+    lo, hi = GOLDEN["w0_share_G1_rank32"]["range"]
+    assert lo < w0 / total < hi
+    assert s_bytes / total < 0.01
+    assert footprint.theta_bytes(fam, L, 1, 4) - footprint.theta_bytes(fam, L, 1, 0) < total - w0
