@@ -69,7 +69,7 @@ def test_stacked_validation(L):
     assert L.wl_stacked_forward(FAKE, 1, 16, arr, P, None) == 3
     assert L.wl_stacked_forward(FAKE, 1, 16, arr, 0, None) == 1
     assert L.wl_stacked_forward(FAKE, 1, 16, None, 1, None) == 1
-    # the decode path serves at most 4 tokens
+    # the decode path serves at most WL_DECODE_MAX_M tokens
     assert L.wl_forward_ex(FAKE, wl.DECODE_MAX_M + 1, 16, arr, 1, wl.PATHS["decode"], None) == 3
     assert L.wl_forward_ex(FAKE, 1, 16, arr, 1, 7, None) == 1
 
@@ -77,3 +77,21 @@ def test_stacked_validation(L):
 def test_wait_probe_rejects_bad_limit(L):
     assert L.wl_wait_probe(0, None) == 1
     assert L.wl_wait_probe(2_000_000_000, None) == 1
+
+
+def test_materialize_validation(L):
+    def mat(W0=FAKE, s=FAKE, U=FAKE, V=FAKE, out=FAKE, N=8, K=16, r=4):
+        return L.wl_materialize_weight(W0, s, U, V, out, N, K, r, None)
+
+    assert mat(N=-1) == 1
+    assert mat(K=-1) == 1
+    assert mat(r=-1) == 1
+    assert mat(r=wl.MAX_RANK + 1) == 3
+    assert mat(W0=None) == 1
+    assert mat(s=None) == 1
+    assert mat(out=None) == 1
+    assert mat(U=None) == 1                  # r > 0 needs U and V
+    assert mat(V=None) == 1
+    # empty weights are a no-op and touch nothing
+    assert mat(N=0, W0=None, s=None, U=None, V=None, out=None) == 0
+    assert mat(K=0, W0=None, s=None, U=None, V=None, out=None) == 0
