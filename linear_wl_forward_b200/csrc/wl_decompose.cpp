@@ -19,13 +19,19 @@
 
 namespace {
 
+constexpr int kJacobiMaxSweeps = 80;
+
 // A is m x n column-major (n <= m).  On return its columns are mutually
-// orthogonal (A_in Q) and Q (n x n, column-major) holds the rotations.
-void jacobi_orthogonalize(std::vector<double> &A, int m, int n, std::vector<double> &Q) {
+// orthogonal (A_in Q) and Q (n x n, column-major) holds the rotations.  A pair
+// counts as orthogonal once |<a_i, a_j>| <= tol ||a_i|| ||a_j||, tol = m times
+// the fp64 unit roundoff (the rounding level of the length-m dot product
+// itself; a tighter test can keep rotating on rounding noise).  Returns false
+// if a sweep still rotated after kJacobiMaxSweeps sweeps.
+bool jacobi_orthogonalize(std::vector<double> &A, int m, int n, std::vector<double> &Q) {
     Q.assign((size_t)n * n, 0.0);
     for (int i = 0; i < n; ++i) Q[(size_t)i * n + i] = 1.0;
-    const double eps = 1e-15;
-    for (int sweep = 0; sweep < 80; ++sweep) {
+    const double eps = std::max(1e-15, (double)m * 1.1102230246251565e-16);
+    for (int sweep = 0; sweep < kJacobiMaxSweeps; ++sweep) {
         bool rotated = false;
         for (int i = 0; i < n - 1; ++i) {
             double *ai = &A[(size_t)i * m];
@@ -56,15 +62,18 @@ void jacobi_orthogonalize(std::vector<double> &A, int m, int n, std::vector<doub
                 }
             }
         }
-        if (!rotated) break;
+        if (!rotated) return true;
     }
+    return false;
 }
 
 // Rank-r truncated SVD of R (N x K, row-major): U = P_r S_r (N x r), V = Q_r (K x r).
-void truncated_svd(const std::vector<double> &R, int N, int K, int r, double *U, double *V) {
+// Returns false if the Jacobi iteration did not converge (the factors are
+// then those of the last sweep).
+bool truncated_svd(const std::vector<double> &R, int N, int K, int r, double *U, double *V) {
     std::fill(U, U + (size_t)N * r, 0.0);
     std::fill(V, V + (size_t)K * r, 0.0);
-    if (r == 0) return;
+    if (r == 0) return true;
     const bool cols_are_k = K <= N;  // orthogonalise the K columns of R, else the N columns of R^T
     const int m = cols_are_k ? N : K, n = cols_are_k ? K : N;
     std::vector<double> A((size_t)m * n);
@@ -76,7 +85,7 @@ void truncated_svd(const std::vector<double> &R, int N, int K, int r, double *U,
                 A[(size_t)a * m + b] = R[(size_t)a * K + b];  // column a of R^T
         }
     std::vector<double> Q;
-    jacobi_orthogonalize(A, m, n, Q);
+    const bool converged = jacobi_orthogonalize(A, m, n, Q);
     std::vector<double> sigma(n);
     for (int i = 0; i < n; ++i) {
         double ss = 0;
@@ -103,6 +112,7 @@ void truncated_svd(const std::vector<double> &R, int N, int K, int r, double *U,
             for (int b = 0; b < K; ++b) V[(size_t)b * r + c] = col[b] / sg;
         }
     }
+    return converged;
 }
 
 double rel_err_fp64(const float *W, const float *W0, const float *s, const float *U, const float *V,
@@ -175,6 +185,7 @@ wl_status decompose_impl(const float *W, int L, int N, int K, int G, int r, cons
             }
         };
         // U_l V_l^T = rank-r truncated SVD of W_l - diag(s_l) W0_b
+        bool converged = true;
         auto fit_delta = [&](int l) {
             if (r == 0) return;
             const float *w = W + (size_t)l * NK;
@@ -182,7 +193,7 @@ wl_status decompose_impl(const float *W, int L, int N, int K, int G, int r, cons
             for (int n = 0; n < N; ++n)
                 for (int k = 0; k < K; ++k)
                     R[(size_t)n * K + k] = (double)w[(size_t)n * K + k] - sd[(size_t)l * N + n] * b0[(size_t)n * K + k];
-            truncated_svd(R, N, K, r, &Ud[(size_t)l * N * r], &Vd[(size_t)l * K * r]);
+            if (!truncated_svd(R, N, K, r, &Ud[(size_t)l * N * r], &Vd[(size_t)l * K * r])) converged = false;
         };
         for (int l = 0; l < L; ++l) {
             fit_scales(l, false);
@@ -221,6 +232,7 @@ wl_status decompose_impl(const float *W, int L, int N, int K, int G, int r, cons
                 rel_err[l] = rel_err_fp64(W + (size_t)l * NK, W0 + (size_t)band[l] * NK, s + (size_t)l * N,
                                           r > 0 ? U + (size_t)l * N * r : nullptr,
                                           r > 0 ? V + (size_t)l * K * r : nullptr, N, K, r);
+        if (!converged) return WL_ERR_NOT_CONVERGED;
     } catch (const std::bad_alloc &) {
         return WL_ERR_NOMEM;
     }

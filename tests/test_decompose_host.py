@@ -96,3 +96,26 @@ def test_als_rejects_negative_rounds():
     W = np.zeros((2, 3, 4), np.float32)
     with pytest.raises(wl.WLError):
         wl.decompose(W, 1, 1, als_iters=-1)
+
+
+def test_gemma3_shape_matches_oracle_and_converges():
+    """One Gemma-3-1B-shaped family at a size the host SVD meets in practice
+    (two layers of 256 x 1152, one band, rank 16): the Jacobi iteration
+    converges (no WL_ERR_NOT_CONVERGED) and the bundle matches the numpy
+    oracle's (W0, s, U V^T and the errors)."""
+    import time
+
+    rng = np.random.default_rng(11)
+    W = (0.02 * rng.standard_normal((2, 256, 1152))).astype(np.float32)
+    t0 = time.perf_counter()
+    W0, s, U, V, err = wl.decompose(W, 1, 16)
+    assert time.perf_counter() - t0 < 120
+    oW0, os_, oU, oV = oracle.decompose(W.astype(np.float64), 1, 16)
+    assert np.allclose(W0, oW0, atol=1e-7)
+    assert np.allclose(s, os_, atol=1e-5)
+    for l in range(2):
+        uv = U[l].astype(np.float64) @ V[l].astype(np.float64).T
+        ouv = oU[l] @ oV[l].T
+        assert np.max(np.abs(uv - ouv)) <= 1e-4 * np.max(np.abs(ouv))
+        oe = oracle.relative_frobenius_error(W[l], oW0[0], os_[l], oU[l], oV[l])
+        assert abs(err[l] - oe) < 1e-5
