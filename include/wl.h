@@ -34,8 +34,18 @@
  *    are reproducible run to run.
  *  - Errors are returned, never aborted on: argument problems are detected on
  *    the host before anything is launched; launch failures give WL_ERR_CUDA; a
- *    device-side wait that exceeded its time limit is reported later by
- *    wl_last_device_status().
+ *    device-side wait that exceeded its time limit (2 s, see
+ *    wl_set_wait_limit) is reported later by wl_last_device_status().  A call
+ *    whose wait gave up leaves its outputs partly unwritten and may leave a
+ *    grid-wide arrival count set, so the results of the calls issued after it
+ *    are undefined until wl_last_device_status() has returned the error (it
+ *    clears the counts).
+ *  - Some kernels wait for one another's CTAs inside one launch (the decode
+ *    kernel's grid-wide V^T x exchange; the GEMM's K-range sums are collected
+ *    by the last CTA to arrive, without waiting).  Those launches never have
+ *    more CTAs than the SMs can hold at once, so on a GPU shared with other
+ *    processes a CTA that cannot become resident within the wait limit makes
+ *    the call fail with WL_ERR_TIMEOUT instead of hanging.
  */
 #ifndef WL_H_
 #define WL_H_
@@ -56,7 +66,8 @@ typedef enum {
     WL_ERR_UNSUPPORTED = 3, /* r > WL_MAX_RANK, P > WL_MAX_PROJ, no sm_100 device */
     WL_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed      */
     WL_ERR_TIMEOUT = 5,     /* a device-side wait gave up (see wl_last_device_status) */
-    WL_ERR_NOMEM = 6        /* scratch pool could not grow                          */
+    WL_ERR_NOMEM = 6,       /* scratch pool could not grow                          */
+    WL_ERR_NOT_CONVERGED = 7 /* host SVD hit its sweep limit (outputs are filled)   */
 } wl_status;
 
 #define WL_MAX_RANK 1024
@@ -75,14 +86,19 @@ typedef struct {
     int r;             /* rank of the delta, 0 <= r <= WL_MAX_RANK     */
 } wl_proj;
 
-/* Which kernels a forward call uses.  WL_PATH_AUTO takes the decode kernel for
+/* Which kernels a forward call uses.  WL_PATH_AUTO takes a decode kernel for
  * M <= 4, and for M <= WL_DECODE_MAX_M when the call's projections total fewer
- * than 8192 output rows; otherwise the tensor-core GEMM.  The others exist so
- * tests and benchmarks can exercise each kernel on any shape. */
+ * than 8192 output rows; otherwise the tensor-core GEMM.  Of the two decode
+ * kernels it takes the row-stream one whenever the call fits it (short calls:
+ * at most four 16-row blocks of W0 per SM, every rank <= 64 and a multiple of
+ * 8, U and V 16-byte aligned), else the weight-streaming one.  The others
+ * exist so tests and benchmarks can exercise each kernel on any shape. */
 typedef enum {
     WL_PATH_AUTO = 0,
     WL_PATH_DECODE = 1, /* weight-streaming kernel (bulk copies + warp MMA), 1 <= M <= WL_DECODE_MAX_M */
-    WL_PATH_GEMM = 2    /* tcgen05 tensor-core GEMM with the fused low-rank epilogue */
+    WL_PATH_GEMM = 2,   /* tcgen05 tensor-core GEMM with the fused low-rank epilogue */
+    WL_PATH_ROWS = 3    /* row-stream decode kernel (register-fed warp MMA, K split over CTA
+                           clusters) for short calls; WL_ERR_UNSUPPORTED for calls it does not fit */
 } wl_path;
 
 #define WL_DECODE_MAX_M 16
@@ -119,9 +135,40 @@ wl_status wl_stacked_forward(const wl_bf16 *x, int M, int K, const wl_proj *proj
                              int P, void *stream);
 
 /* wl_stacked_forward with an explicit kernel choice (see wl_path).
- * WL_PATH_DECODE requires M <= WL_DECODE_MAX_M (else WL_ERR_UNSUPPORTED). */
+ * WL_PATH_DECODE and WL_PATH_ROWS require M <= WL_DECODE_MAX_M (else
+ * WL_ERR_UNSUPPORTED); WL_PATH_ROWS also the limits of that kernel. */
 wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
                         wl_path path, void *stream);
+
+/* A device range for wl_stacked_forward_prefetch. */
+typedef struct {
+    const void *ptr; /* device address (any alignment)                   */
+    size_t bytes;    /* length; 0 is allowed and ignored                 */
+} wl_range;
+
+#define WL_MAX_PREFETCH 32
+
+/* wl_forward_ex that also pulls `prefetch` (a HOST array of n ranges of
+ * device memory, 0 <= n <= WL_MAX_PREFETCH; NULL iff n == 0) into L2 while
+ * the call runs.  A decode step runs a fixed sequence of projections whose
+ * weights do not change, so each call can name the weights of the call (or
+ * calls) that follow it: those then start from L2 instead of HBM, and the
+ * HBM stream of one call overlaps the arithmetic and epilogue of the one
+ * before.  The pages name the cost this hides ("Quality (Gemma 4 31B)",
+ * "Kernel optimizations": kernel launch overhead at batch-size-1 decode, and
+ * the custom op being memory-bound at small dimensions).
+ * Each range is trimmed to its 16-byte-aligned interior (so no byte outside
+ * it is touched); the call's kernels share the bytes out over their CTAs and
+ * issue them at their start, before waiting for the previous kernel in the
+ * stream.  A prefetch moves data into L2 only, and L2 is coherent for the
+ * whole device, so it never changes any result: ranges may hold anything,
+ * including buffers other kernels are writing.  Keep the total well below
+ * the 126 MB L2 (a few calls' weights).  Errors: those of wl_forward_ex;
+ * WL_ERR_INVALID_ARG for n < 0, n > WL_MAX_PREFETCH, a NULL array with
+ * n > 0, or a NULL range pointer with bytes > 0. */
+wl_status wl_stacked_forward_prefetch(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                                      wl_path path, const wl_range *prefetch, int n,
+                                      void *stream);
 
 /* wl_linear_forward for callers that cannot allocate device memory while they
  * run: code living inside a pre-planned memory arena (an inference engine
@@ -147,10 +194,22 @@ wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, in
  *    Calls that overlap on the GPU (different streams or host threads) race on
  *    the array: serialise them.
  *  - A device-side wait that times out here is recorded in the array's own
- *    status word, not in the word wl_last_device_status() reads. */
+ *    status word, which wl_noalloc_last_status() reads (not
+ *    wl_last_device_status()); each call clears the array's arrival counts
+ *    before its kernel runs, and the status word keeps the first error until
+ *    it is read. */
 wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *W0, const float *s,
                                     const wl_bf16 *U, const wl_bf16 *V, wl_bf16 *y,
                                     int M, int N, int K, int r, void *stream);
+
+/* Synchronises `stream`, then returns the status word of
+ * wl_linear_forward_noalloc's array on the current device: WL_OK, or the
+ * first error one of its calls recorded (WL_ERR_TIMEOUT from a device-side
+ * wait that gave up) since the word was last read with an error.  After an
+ * error it clears the array's status word and arrival counts.  Makes no
+ * allocation; like the forward, its first call on a device looks up the
+ * array's address. */
+wl_status wl_noalloc_last_status(void *stream);
 
 /* Host-side decomposition of L dense layer weights into theta bundles
  * ("Quality", "Why sharing fails": band-mean W0, per-row scale s, low-rank
@@ -169,9 +228,14 @@ wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *W0, const f
  *   rel_err (out) : host, L doubles, may be NULL -- relative Frobenius error
  *                   of diag(s) W0 + U V^T against W_l, in fp64 from the fp32
  *                   factors
- * Computes in fp64 on the calling thread, synchronously.  Returns
- * WL_ERR_INVALID_ARG for null pointers, L, N, K, G < 1, r < 0 or a band index
- * outside [0, G); WL_ERR_NOMEM if host memory runs out. */
+ * Computes in fp64 on the calling thread, synchronously; the SVD is a
+ * one-sided Jacobi iteration, stopped when every column pair is orthogonal to
+ * the rounding level of its dot products (m times the fp64 unit roundoff, m
+ * the column length) or after 80 sweeps.  Returns WL_ERR_INVALID_ARG for null
+ * pointers, L, N, K, G < 1, r < 0 or a band index outside [0, G);
+ * WL_ERR_NOMEM if host memory runs out; WL_ERR_NOT_CONVERGED (every output
+ * still written, from the last sweep) if some layer's iteration reached the
+ * sweep limit. */
 wl_status wl_decompose(const float *W, int L, int N, int K, int G, int r,
                        const int *band_of_layer, float *W0, float *s, float *U,
                        float *V, double *rel_err);
@@ -268,6 +332,27 @@ typedef struct {
 wl_status wl_describe_decode_plan(int M, int K, const wl_proj *projs, int P, int num_sms,
                                   wl_decode_plan *out);
 
+/* The row-stream kernel's host-side plan for a call (see WL_PATH_ROWS), made
+ * without a GPU; the pointers in `projs` are checked for NULL and alignment
+ * only.  Output rows are cut into 16-row blocks, the blocks of each
+ * projection into row groups of at most nb_max blocks, and each row group is
+ * owned by a cluster of `cluster` CTAs that split K into slices of
+ * k_slice columns. */
+typedef struct {
+    int grid;         /* CTAs (row groups x cluster), at most num_sms        */
+    int cluster;      /* CTAs per cluster (1, 2 or 4)                        */
+    int row_groups;   /* clusters                                            */
+    int nb_max;       /* largest number of 16-row blocks of one row group    */
+    int k_slice;      /* K columns per CTA of a cluster                      */
+    long long smem_bytes; /* dynamic shared memory per CTA                   */
+} wl_rows_plan;
+
+/* Fills *out for the call on a GPU with num_sms SMs.  Returns
+ * WL_ERR_UNSUPPORTED for calls the row-stream kernel does not take, and the
+ * argument errors of wl_stacked_forward. */
+wl_status wl_describe_rows_plan(int M, int K, const wl_proj *projs, int P, int num_sms,
+                                wl_rows_plan *out);
+
 /* Static description of a status code. */
 const char *wl_status_string(wl_status status);
 
@@ -275,6 +360,14 @@ const char *wl_status_string(wl_status status);
  * word: WL_OK, or the first error a kernel recorded since the last call (for
  * example WL_ERR_TIMEOUT from a wait that gave up). */
 wl_status wl_last_device_status(void *stream);
+
+/* Sets the time limit of every device-side wait of the forward calls issued
+ * afterwards, on every device (limit_ns in nanoseconds, 1 ..  1e10; 0 restores
+ * the default of 2 s).  For tests of the time-out path: a short limit makes
+ * waits give up (WL_ERR_TIMEOUT via wl_last_device_status) instead of
+ * waiting; every wait is bounded either way.  Returns WL_ERR_INVALID_ARG
+ * outside that range. */
+wl_status wl_set_wait_limit(long long limit_ns);
 
 /* Launches one probe kernel that waits on a device flag nothing ever sets,
  * giving up after `limit_ns` nanoseconds and recording WL_ERR_TIMEOUT in the

@@ -12,9 +12,11 @@ import os
 
 __all__ = [
     "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
-    "materialize_weight", "describe_decode_plan", "DecodePlan", "quantize_nvfp4",
+    "prefetch_ranges", "MAX_PREFETCH",
+    "materialize_weight", "describe_decode_plan", "DecodePlan", "describe_rows_plan", "RowsPlan",
+    "quantize_nvfp4",
     "decompose",
-    "relative_frobenius_error", "last_device_status", "wait_probe", "PATHS",
+    "relative_frobenius_error", "last_device_status", "wait_probe", "set_wait_limit", "PATHS",
     "DECODE_MAX_M", "MAX_RANK", "MAX_PROJ", "STATUS",
 ]
 
@@ -22,11 +24,12 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwl.so")
 
 STATUS = {0: "WL_OK", 1: "WL_ERR_INVALID_ARG", 2: "WL_ERR_ALIGNMENT", 3: "WL_ERR_UNSUPPORTED",
-          4: "WL_ERR_CUDA", 5: "WL_ERR_TIMEOUT", 6: "WL_ERR_NOMEM"}
-PATHS = {"auto": 0, "decode": 1, "gemm": 2}
+          4: "WL_ERR_CUDA", 5: "WL_ERR_TIMEOUT", 6: "WL_ERR_NOMEM", 7: "WL_ERR_NOT_CONVERGED"}
+PATHS = {"auto": 0, "decode": 1, "gemm": 2, "rows": 3}
 DECODE_MAX_M = 16
 MAX_RANK = 1024
 MAX_PROJ = 8
+MAX_PREFETCH = 32
 
 
 class WLError(RuntimeError):
@@ -40,6 +43,16 @@ class _Proj(ctypes.Structure):
     _fields_ = [("W0", ctypes.c_void_p), ("s", ctypes.c_void_p), ("U", ctypes.c_void_p),
                 ("V", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int),
                 ("r", ctypes.c_int)]
+
+
+class _Range(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("bytes", ctypes.c_size_t)]
+
+
+class RowsPlan(ctypes.Structure):
+    """wl_rows_plan of include/wl.h."""
+    _fields_ = [("grid", ctypes.c_int), ("cluster", ctypes.c_int), ("row_groups", ctypes.c_int),
+                ("nb_max", ctypes.c_int), ("k_slice", ctypes.c_int), ("smem_bytes", ctypes.c_longlong)]
 
 
 class DecodePlan(ctypes.Structure):
@@ -66,11 +79,14 @@ def lib():
         L.wl_linear_forward.argtypes = [vp] * 6 + [ci] * 4 + [vp]
         L.wl_stacked_forward.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, vp]
         L.wl_forward_ex.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, ci, vp]
+        L.wl_stacked_forward_prefetch.argtypes = [vp, ci, ci, ctypes.POINTER(_Proj), ci, ci,
+                                                  ctypes.POINTER(_Range), ci, vp]
         L.wl_decompose.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp]
         L.wl_decompose_als.argtypes = [vp, ci, ci, ci, ci, ci, vp, ci, vp, vp, vp, vp, vp]
         L.wl_materialize_weight.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, vp]
         L.wl_describe_decode_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci,
                                               ctypes.POINTER(DecodePlan)]
+        L.wl_describe_rows_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci, ctypes.POINTER(RowsPlan)]
         L.wl_quantize_nvfp4.argtypes = [vp, ci, ci, ctypes.c_float, vp, vp, ctypes.POINTER(ctypes.c_float)]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
         L.wl_relative_frobenius_error.restype = ctypes.c_double
@@ -78,10 +94,14 @@ def lib():
         L.wl_status_string.restype = ctypes.c_char_p
         L.wl_last_device_status.argtypes = [vp]
         L.wl_wait_probe.argtypes = [cll, vp]
+        L.wl_set_wait_limit.argtypes = [cll]
+        L.wl_noalloc_last_status.argtypes = [vp]
         L.wl_version.restype = ci
-        for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_decompose", "wl_decompose_als",
-                     "wl_materialize_weight", "wl_describe_decode_plan", "wl_quantize_nvfp4",
-                     "wl_last_device_status", "wl_wait_probe"):
+        for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_stacked_forward_prefetch",
+                     "wl_decompose", "wl_decompose_als",
+                     "wl_materialize_weight", "wl_describe_decode_plan", "wl_describe_rows_plan",
+                     "wl_quantize_nvfp4",
+                     "wl_last_device_status", "wl_wait_probe", "wl_set_wait_limit", "wl_noalloc_last_status"):
             getattr(L, name).restype = ci
         _lib = L
     return _lib
@@ -137,9 +157,33 @@ def linear_forward(x, W0, s, U, V, y=None, stream=None, path="auto"):
                            path=path)[0]
 
 
-def stacked_forward(x, projs, ys=None, stream=None, path="auto"):
+def prefetch_ranges(items):
+    """wl_range array for wl_stacked_forward_prefetch from CUDA tensors (their
+    whole storage from data_ptr) and/or (device address, bytes) pairs; None
+    entries are skipped."""
+    import torch
+
+    ranges = []
+    for it in items:
+        if it is None:
+            continue
+        if isinstance(it, torch.Tensor):
+            if not it.is_cuda:
+                raise TypeError("prefetch tensors must be CUDA tensors")
+            ranges.append((it.data_ptr(), it.numel() * it.element_size()))
+        else:
+            ptr, nbytes = it
+            ranges.append((int(ptr), int(nbytes)))
+    if len(ranges) > MAX_PREFETCH:
+        raise ValueError(f"at most {MAX_PREFETCH} prefetch ranges, got {len(ranges)}")
+    return (_Range * max(len(ranges), 1))(*[_Range(p, n) for p, n in ranges]), len(ranges)
+
+
+def stacked_forward(x, projs, ys=None, stream=None, path="auto", prefetch=None):
     """Several projections (W0_p, s_p, U_p, V_p) against one shared x in one
-    call.  Returns the list of y_p (M x N_p bf16)."""
+    call.  Returns the list of y_p (M x N_p bf16).  `prefetch`: tensors (or
+    (address, bytes) pairs) to pull into L2 while the call runs, normally the
+    weights of the call that follows (include/wl.h, wl_stacked_forward_prefetch)."""
     import torch
 
     M, K = x.shape
@@ -149,8 +193,13 @@ def stacked_forward(x, projs, ys=None, stream=None, path="auto"):
     arr = (_Proj * len(projs))(*[_make_proj(W0, s, U, V, y, M, K)
                                  for (W0, s, U, V), y in zip(projs, ys)])
     xp = _dev_ptr(x, torch.bfloat16, "x", (M, K))
-    _check(lib().wl_forward_ex(xp, M, K, arr, len(projs), PATHS[path], _stream_handle(stream)),
-           "wl_forward_ex")
+    if prefetch:
+        rng, n = prefetch_ranges(prefetch)
+        _check(lib().wl_stacked_forward_prefetch(xp, M, K, arr, len(projs), PATHS[path], rng, n,
+                                                 _stream_handle(stream)), "wl_stacked_forward_prefetch")
+    else:
+        _check(lib().wl_forward_ex(xp, M, K, arr, len(projs), PATHS[path], _stream_handle(stream)),
+               "wl_forward_ex")
     return ys
 
 
@@ -165,7 +214,7 @@ class PreparedForward:
     replaced (in-place writes to x and the weights between calls are fine).
     """
 
-    def __init__(self, x, projs, ys=None, path="auto"):
+    def __init__(self, x, projs, ys=None, path="auto", prefetch=None):
         import torch
 
         M, K = x.shape
@@ -173,22 +222,25 @@ class PreparedForward:
             ys = [torch.empty(M, W0.shape[0], dtype=torch.bfloat16, device=x.device)
                   for (W0, _, _, _) in projs]
         self.ys = ys
-        self._keep = (x, projs, ys)
+        self._keep = (x, projs, ys, prefetch)
         self._arr = (_Proj * len(projs))(*[_make_proj(W0, s, U, V, y, M, K)
                                            for (W0, s, U, V), y in zip(projs, ys)])
+        self._rng, self._nrng = prefetch_ranges(prefetch or [])
         self._args = (_dev_ptr(x, torch.bfloat16, "x", (M, K)), M, K, self._arr, len(projs), PATHS[path])
-        self._fn = lib().wl_forward_ex
+        self._fn = lib().wl_stacked_forward_prefetch
 
     def __call__(self, stream=None):
         xp, M, K, arr, P, path = self._args
-        _check(self._fn(xp, M, K, arr, P, path, _stream_handle(stream)), "wl_forward_ex")
+        _check(self._fn(xp, M, K, arr, P, path, self._rng, self._nrng, _stream_handle(stream)),
+               "wl_stacked_forward_prefetch")
         return self.ys
 
 
-def prepare_stacked(x, projs, ys=None, path="auto") -> PreparedForward:
+def prepare_stacked(x, projs, ys=None, path="auto", prefetch=None) -> PreparedForward:
     """``stacked_forward`` with its argument checks done once: returns a
-    callable that issues the forward (see PreparedForward)."""
-    return PreparedForward(x, projs, ys, path)
+    callable that issues the forward (see PreparedForward).  `prefetch` as in
+    ``stacked_forward``."""
+    return PreparedForward(x, projs, ys, path, prefetch)
 
 
 def materialize_weight(W0, s, U, V, out=None, stream=None):
@@ -246,9 +298,37 @@ def describe_decode_plan(M: int, K: int, projs, num_sms: int = 148) -> dict:
     return {name: getattr(out, name) for name, _ in DecodePlan._fields_}
 
 
+def _stand_in_projs(projs):
+    arr = (_Proj * len(projs))()
+    for i, q in enumerate(projs):
+        N, r = q[0], q[1]
+        off = q[2] if len(q) > 2 else 0
+        base = (i + 1) << 32
+        arr[i] = _Proj(base, base + (1 << 28), (base + (2 << 28) + off) if r else None,
+                       (base + (3 << 28) + off) if r else None, base + (4 << 28), N, r)
+    return arr
+
+
+def describe_rows_plan(M: int, K: int, projs, num_sms: int = 148) -> dict:
+    """The row-stream kernel's host-side plan for a call, made without a GPU
+    (``projs`` as in ``describe_decode_plan``).  Raises WLError (code 3) for
+    calls the kernel does not take."""
+    arr = _stand_in_projs(projs)
+    out = RowsPlan()
+    _check(lib().wl_describe_rows_plan(M, K, arr, len(projs), num_sms, ctypes.byref(out)),
+           "wl_describe_rows_plan")
+    return {name: getattr(out, name) for name, _ in RowsPlan._fields_}
+
+
 def last_device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device status word."""
     return lib().wl_last_device_status(_stream_handle(stream))
+
+
+def set_wait_limit(limit_ns: int):
+    """Time limit of the device-side waits of later forward calls (0: the
+    default, 2 s); for tests of the time-out path."""
+    _check(lib().wl_set_wait_limit(int(limit_ns)), "wl_set_wait_limit")
 
 
 def wait_probe(limit_ns: int, stream=None):

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <memory>
@@ -78,6 +79,7 @@ wl_status make_map(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per device-side wait
 constexpr int kMaxDevices = 64;
+std::atomic<unsigned long long> g_wait_limit_ns{kWaitLimitNs};
 
 enum Slot {
     kSlotT = 0,
@@ -154,7 +156,7 @@ wl_status validate(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, 
     if (!projs) return WL_ERR_INVALID_ARG;
     if (P < 1 || P > WL_MAX_PROJ) return P < 1 ? WL_ERR_INVALID_ARG : WL_ERR_UNSUPPORTED;
     if (M < 0 || K < 0) return WL_ERR_INVALID_ARG;
-    if (path != WL_PATH_AUTO && path != WL_PATH_DECODE && path != WL_PATH_GEMM)
+    if (path != WL_PATH_AUTO && path != WL_PATH_DECODE && path != WL_PATH_GEMM && path != WL_PATH_ROWS)
         return WL_ERR_INVALID_ARG;
     for (int i = 0; i < P; ++i) {
         const wl_proj &q = projs[i];
@@ -172,11 +174,31 @@ wl_status validate(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, 
         for (int i = 0; i < P; ++i)
             if (projs[i].N > 0 && !aligned16(projs[i].W0)) return WL_ERR_ALIGNMENT;
     }
-    if (path == WL_PATH_DECODE && M > WL_DECODE_MAX_M) return WL_ERR_UNSUPPORTED;
+    if ((path == WL_PATH_DECODE || path == WL_PATH_ROWS) && M > WL_DECODE_MAX_M) return WL_ERR_UNSUPPORTED;
     return WL_OK;
 }
 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// The prefetch ranges of a call, each trimmed to its 16-byte-aligned interior
+// (empty ones dropped).  Pure host code.
+wl_status build_prefetch(const wl_range *ranges, int n, PrefetchList &pf) {
+    std::memset(&pf, 0, sizeof pf);
+    if (n < 0 || n > WL_MAX_PREFETCH || (n > 0 && !ranges)) return WL_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        if (ranges[i].bytes == 0) continue;
+        if (!ranges[i].ptr) return WL_ERR_INVALID_ARG;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(ranges[i].ptr);
+        const uintptr_t lo = (a + 15) & ~uintptr_t(15);
+        const uintptr_t hi = (a + ranges[i].bytes) & ~uintptr_t(15);
+        if (hi <= lo) continue;
+        pf.ptr[pf.n] = reinterpret_cast<const uint8_t *>(lo);
+        pf.bytes[pf.n] = hi - lo;
+        pf.total += hi - lo;
+        ++pf.n;
+    }
+    return WL_OK;
+}
 
 // WL_PATH_AUTO: the weight-streaming decode kernel for up to 4 tokens, and
 // for up to WL_DECODE_MAX_M tokens when the call is narrow (its projections
@@ -222,7 +244,6 @@ bool build_decode_params(const wl_bf16 *x, int M, int K, const wl_proj *projs, i
     dp.a.K = K;
     dp.a.t_ld = t_off;
     dp.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-    dp.a.timeout_ns = kWaitLimitNs;
     return true;
 }
 
@@ -258,7 +279,7 @@ constexpr size_t kDecodeCacheMax = 4096;
 std::unordered_map<DecodeKey, std::unique_ptr<DecodeEntry>, DecodeKeyHash> g_decode_cache[kMaxDevices];
 
 wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
-                     cudaStream_t stream) {
+                     const PrefetchList &pf, cudaStream_t stream) {
     DecodeKey key;
     std::memset(&key, 0, sizeof key);  // padding bytes take part in the comparison
     key.x = x;
@@ -284,6 +305,8 @@ wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_
     const DecodePlan &plan = e.plan;
     dp.a.status = pool.words;
     dp.a.sync = reinterpret_cast<unsigned int *>(pool.words + 8);
+    dp.a.timeout_ns = wait_limit_ns();
+    dp.pf = pf;
     if (plan.tpart_bytes) {
         void *tp = nullptr;
         wl_status st = scratch(pool, kSlotTPart, plan.tpart_bytes, &tp);
@@ -293,8 +316,47 @@ wl_status run_decode(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_
     return from_cuda(launch_decode(dp, plan, stream));
 }
 
+// Row-stream plans of recent calls, keyed like the decode plans (no tensor
+// maps: planning is cheap, but a decode step repeats its calls).
+struct RowsEntry {
+    RowsParams rp;
+    wl_status status;  // WL_OK or WL_ERR_UNSUPPORTED (the call does not fit the kernel)
+};
+std::unordered_map<DecodeKey, std::unique_ptr<RowsEntry>, DecodeKeyHash> g_rows_cache[kMaxDevices];
+
+// Returns WL_ERR_UNSUPPORTED (launching nothing) if the call does not fit the
+// row-stream kernel.
+wl_status run_rows(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                   const PrefetchList &pf, cudaStream_t stream) {
+    DecodeKey key;
+    std::memset(&key, 0, sizeof key);
+    key.x = x;
+    key.M = M;
+    key.K = K;
+    key.P = P;
+    std::memcpy(key.projs, projs, sizeof(wl_proj) * P);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WL_ERR_CUDA;
+    auto &cache = g_rows_cache[dev];
+    auto it = cache.find(key);
+    if (it == cache.end()) {
+        if (cache.size() >= kDecodeCacheMax) cache.clear();
+        auto e = std::make_unique<RowsEntry>();
+        e->status = plan_rows(e->rp, M, K, projs, P, pool.num_sms);
+        if (e->status != WL_OK && e->status != WL_ERR_UNSUPPORTED) return e->status;
+        it = cache.emplace(key, std::move(e)).first;
+    }
+    RowsEntry &e = *it->second;
+    if (e.status != WL_OK) return e.status;
+    e.rp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    e.rp.status = pool.words;
+    e.rp.timeout_ns = wait_limit_ns();
+    e.rp.pf = pf;
+    return from_cuda(launch_rows(e.rp, stream));
+}
+
 wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
-                   cudaStream_t stream) {
+                   const PrefetchList &pf, cudaStream_t stream) {
     // Column layout of T: each projection with r > 0 gets round_up(r, 64) columns.
     int t_cols = 0;
     int t_col[kMaxSeg] = {};
@@ -348,7 +410,7 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
         tp.kb_split = (K + kGemmBK - 1) / kGemmBK;
         set_gemm_stages(tp);
         tp.status = pool.words;
-        tp.timeout_ns = kWaitLimitNs;
+        tp.timeout_ns = wait_limit_ns();
         if (launch_gemm(tp, pool.num_sms, stream) != cudaSuccess) return WL_ERR_CUDA;
     }
 
@@ -451,14 +513,17 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
     }
     set_gemm_stages(gp);
     gp.status = pool.words;
-    gp.timeout_ns = kWaitLimitNs;
+    gp.timeout_ns = wait_limit_ns();
+    gp.pf = pf;
     return from_cuda(launch_gemm(gp, pool.num_sms, stream));
 }
 
 wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, wl_path path,
-                  void *stream_ptr) {
+                  const wl_range *prefetch, int nprefetch, void *stream_ptr) {
     wl_status st = validate(x, M, K, projs, P, path);
     if (st != WL_OK) return st;
+    PrefetchList pf;
+    if ((st = build_prefetch(prefetch, nprefetch, pf)) != WL_OK) return st;
     bool any = false;
     for (int i = 0; i < P; ++i) any = any || projs[i].N > 0;
     if (M == 0 || !any) return WL_OK;
@@ -474,19 +539,33 @@ wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, w
     DevicePool *pool = nullptr;
     if ((st = pool_for_current_device(&pool)) != WL_OK) return st;
     if (path == WL_PATH_AUTO && auto_decode(M, projs, P)) {
-        // The decode kernel declines shapes it cannot hold (before launching
-        // anything); those go to the tensor-core GEMM.
-        st = run_decode(*pool, x, M, K, projs, P, stream);
-        return st == WL_ERR_UNSUPPORTED ? run_gemm(*pool, x, M, K, projs, P, stream) : st;
+        // Each decode kernel declines shapes it cannot hold (before launching
+        // anything): short calls take the row-stream kernel, the rest the
+        // weight-streaming one, and what neither holds the tensor-core GEMM.
+        st = run_rows(*pool, x, M, K, projs, P, pf, stream);
+        if (st != WL_ERR_UNSUPPORTED) return st;
+        st = run_decode(*pool, x, M, K, projs, P, pf, stream);
+        return st == WL_ERR_UNSUPPORTED ? run_gemm(*pool, x, M, K, projs, P, pf, stream) : st;
     }
-    return path == WL_PATH_DECODE ? run_decode(*pool, x, M, K, projs, P, stream)
-                                  : run_gemm(*pool, x, M, K, projs, P, stream);
+    if (path == WL_PATH_ROWS) return run_rows(*pool, x, M, K, projs, P, pf, stream);
+    return path == WL_PATH_DECODE ? run_decode(*pool, x, M, K, projs, P, pf, stream)
+                                  : run_gemm(*pool, x, M, K, projs, P, pf, stream);
 }
 
 }  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 }  // namespace wl
 
 extern "C" {
+
+wl_status wl_set_wait_limit(long long limit_ns) {
+    if (limit_ns < 0 || limit_ns > 10000000000LL) return WL_ERR_INVALID_ARG;
+    wl::g_wait_limit_ns.store(limit_ns == 0 ? wl::kWaitLimitNs : (unsigned long long)limit_ns,
+                              std::memory_order_relaxed);
+    return WL_OK;
+}
 
 wl_status wl_linear_forward(const wl_bf16 *x, const wl_bf16 *W0, const float *s, const wl_bf16 *U,
                             const wl_bf16 *V, wl_bf16 *y, int M, int N, int K, int r, void *stream) {
@@ -498,17 +577,22 @@ wl_status wl_linear_forward(const wl_bf16 *x, const wl_bf16 *W0, const float *s,
     p.y = y;
     p.N = N;
     p.r = r;
-    return wl::forward(x, M, K, &p, 1, WL_PATH_AUTO, stream);
+    return wl::forward(x, M, K, &p, 1, WL_PATH_AUTO, nullptr, 0, stream);
 }
 
 wl_status wl_stacked_forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
                              void *stream) {
-    return wl::forward(x, M, K, projs, P, WL_PATH_AUTO, stream);
+    return wl::forward(x, M, K, projs, P, WL_PATH_AUTO, nullptr, 0, stream);
 }
 
 wl_status wl_forward_ex(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, wl_path path,
                         void *stream) {
-    return wl::forward(x, M, K, projs, P, path, stream);
+    return wl::forward(x, M, K, projs, P, path, nullptr, 0, stream);
+}
+
+wl_status wl_stacked_forward_prefetch(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                                      wl_path path, const wl_range *prefetch, int n, void *stream) {
+    return wl::forward(x, M, K, projs, P, path, prefetch, n, stream);
 }
 
 const char *wl_status_string(wl_status s) {
@@ -519,7 +603,8 @@ const char *wl_status_string(wl_status s) {
         case WL_ERR_UNSUPPORTED: return "unsupported (rank, projection count, path or device)";
         case WL_ERR_CUDA: return "CUDA error";
         case WL_ERR_TIMEOUT: return "device-side wait timed out";
-        case WL_ERR_NOMEM: return "out of device memory";
+        case WL_ERR_NOMEM: return "out of memory";
+        case WL_ERR_NOT_CONVERGED: return "host SVD did not converge within its sweep limit";
     }
     return "unknown status";
 }
@@ -569,6 +654,23 @@ wl_status wl_describe_decode_plan(int M, int K, const wl_proj *projs, int P, int
     out->v_in_ring = a.v_in_ring;
     out->u_stage = a.u_stage;
     out->lag = a.lag;
+    return WL_OK;
+}
+
+wl_status wl_describe_rows_plan(int M, int K, const wl_proj *projs, int P, int num_sms, wl_rows_plan *out) {
+    if (!out || num_sms < 1) return WL_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof *out);
+    alignas(16) static const unsigned char no_x[16] = {};
+    wl_status st = wl::validate(reinterpret_cast<const wl_bf16 *>(no_x), M, K, projs, P, WL_PATH_ROWS);
+    if (st != WL_OK) return st;
+    wl::RowsParams rp;
+    if ((st = wl::plan_rows(rp, M, K, projs, P, num_sms)) != WL_OK) return st;
+    out->grid = rp.ngroups * rp.c;
+    out->cluster = rp.c;
+    out->row_groups = rp.ngroups;
+    out->nb_max = rp.nb_max;
+    out->k_slice = rp.ks;
+    out->smem_bytes = (long long)rp.smem;
     return WL_OK;
 }
 

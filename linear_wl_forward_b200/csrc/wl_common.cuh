@@ -100,6 +100,12 @@ __device__ __forceinline__ void tma_load_2d(void *dst_smem, const void *tmap, in
         : "memory");
 }
 
+// Bulk prefetch of `bytes` (a multiple of 16) at a 16-byte-aligned global
+// address into L2; nothing lands in shared memory and nothing is waited for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

@@ -61,8 +61,11 @@
 // W0 stream is staged by TMA, the per-row dot products run on the tensor
 // cores, rows are spread evenly over all SMs, and consecutive calls overlap
 // through programmatic dependent launch.
+#include <atomic>
+
 #include "wl_common.cuh"
 #include "wl_internal.h"
+#include "wl_prefetch.cuh"
 
 namespace wl {
 
@@ -990,6 +993,8 @@ __global__ void __launch_bounds__(NTH, SMALL ? 2 : 1) decode_kernel(const __grid
     // the whole ring, less the level that holds V until T's sums are formed
     const uint32_t pre_slots = p.v_in_ring ? (uint32_t)SLOTS - 1u : (uint32_t)SLOTS;
     while (more && issued < pre_slots) issue_next();
+    // the following call's weights into L2, behind this CTA's own copies
+    if (tid == NTH - 32) l2_prefetch_share(P.pf, blockIdx.x, gridDim.x);
     // Output index of this thread in the epilogue of step u (-1: not its turn).
     const int E = (BR * M + 31) / 32;  // warps per epilogue
     auto epi_out = [&](int u) -> int {
@@ -1650,19 +1655,19 @@ static cudaError_t launch_decode_v(const DecodeParams &p, const DecodePlan &plan
     // Opt in to the large shared-memory carve-out once per device: both
     // variants run with all of the SM's shared memory configured, so the
     // compact one can hold two CTAs (of consecutive calls) per SM.
-    static bool attr_done[64] = {};
+    static std::atomic<bool> attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL, FT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kDecodeMaxSmem);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(decode_kernel<NT, XS, SMALL, FT>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.grid);

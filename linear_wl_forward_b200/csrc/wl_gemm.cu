@@ -34,8 +34,11 @@
 // optimizations", GEMM path item 2 (bf16 matmuls accumulate in fp32 on the
 // tensor cores); the pages' GEMM path uses two library matmuls per stack, here
 // the low-rank product rides in the same kernel and the same accumulator pass.
+#include <atomic>
+
 #include "wl_common.cuh"
 #include "wl_internal.h"
+#include "wl_prefetch.cuh"
 
 namespace wl {
 
@@ -133,6 +136,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             prefetch_tmap(&p.tm_b[i]);
             prefetch_tmap(&p.tm_u[i]);
         }
+        l2_prefetch_share(p.pf, blockIdx.x, gridDim.x);  // the following call's weights
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -439,15 +443,15 @@ cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
     const size_t smem = gemm_smem_bytes(p);
     if (p.stages < 2 || p.stages > kGemmMaxStages || smem > 227 * 1024) return cudaErrorInvalidValue;
     // Opt in to the large shared-memory carve-out once per device.
-    static bool attr_done[64] = {};
+    static std::atomic<bool> attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_release);
     }
     if (p.ksplit < 1 || (p.swap && (p.mp < 16 || p.mp > 64 || p.mp % 16 != 0))) return cudaErrorInvalidValue;
     const int units = p.num_tiles * p.ksplit;

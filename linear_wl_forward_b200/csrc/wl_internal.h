@@ -12,6 +12,21 @@ namespace wl {
 
 constexpr int kMaxSeg = WL_MAX_PROJ;
 
+// ------------------------------------------------------------- prefetch ----
+// Device ranges a call's kernels pull into L2 for the calls that follow it
+// (wl_stacked_forward_prefetch): each range is trimmed on the host to its
+// 16-byte-aligned interior, and the CTAs of the launch share the bytes out
+// evenly, in order.
+constexpr int kMaxPrefetch = WL_MAX_PREFETCH;
+constexpr uint32_t kPrefetchPiece = 64 * 1024;  // bytes per bulk prefetch instruction
+
+struct PrefetchList {
+    const uint8_t *ptr[kMaxPrefetch];  // 16-byte aligned
+    uint64_t bytes[kMaxPrefetch];      // multiples of 16
+    uint64_t total;                    // sum of bytes
+    int n;
+};
+
 // --------------------------------------------------------------- decode ----
 // Streaming decode kernel: M <= WL_DECODE_MAX_M tokens.  The projections of a
 // stacked call are concatenated into one list of 16-row blocks.
@@ -82,6 +97,7 @@ struct DecodeArgs {
 
 struct DecodeParams {
     DecodeArgs a;
+    PrefetchList pf;             // read by one thread per CTA, before the wait
     CUtensorMap tm_w[kMaxSeg];   // W0: 2-D {K, N}, box {64, 16}, 128-B swizzle
     CUtensorMap tm_w3[kMaxSeg];  // W0: 3-D {64, N, K/64}, box {64, 16, slot_chunks} (when w3d)
     CUtensorMap tm_u[kMaxSeg];   // U:  2-D {r, N}, box {64, 16} (when u_bulk)
@@ -109,6 +125,56 @@ wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t
 wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                         uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
                         uint32_t b2);
+
+// ----------------------------------------------------------- row stream ----
+// Row-stream decode kernel for short calls (latency-bound: a few MB of
+// weights).  Each CTA owns a group of up to kRowsMaxBlocks 16-row blocks of
+// one projection and, with a cluster of c CTAs, 1/c of K; before the wait for
+// the previous kernel its lanes copy their W0 MMA fragments into shared
+// memory (cp.async) and V and U rows are bulk-copied there, and the partial
+// sums of the c CTAs meet over distributed shared memory.
+constexpr int kRowsWarps = 8;
+constexpr int kRowsThreads = 32 * kRowsWarps;
+constexpr int kRowsKGroup = 32;     // K columns per warp step (two m16n8k16 MMAs)
+constexpr int kRowsMaxBlocks = 4;   // 16-row blocks per CTA
+constexpr int kRowsMaxRank = 64;    // four 16-column tiles of T
+constexpr int kRowsMaxCluster = 4;  // CTAs sharing one row group along K
+constexpr int kRowsXPad = 32;       // elements of padding per staged x row (bank spread)
+
+struct RowsSeg {
+    const __nv_bfloat16 *W0;
+    const float *s;
+    const __nv_bfloat16 *U;
+    const __nv_bfloat16 *V;
+    __nv_bfloat16 *y;
+    int N, r;
+    int grp_begin;  // first row group (cluster) of this projection
+    int nb;         // 16-row blocks per row group (the last group may have fewer)
+};
+
+struct RowsParams {
+    RowsSeg seg[kMaxSeg];
+    int nseg;
+    int M, K;
+    int c;       // CTAs per cluster: the K slices of one row group
+    int ks;      // K columns per slice (a multiple of kRowsKGroup)
+    int ngroups; // row groups (clusters) in the grid
+    int nb_max;  // largest nb over the projections
+    int r_max;
+    // shared memory offsets (bytes) and total
+    uint32_t off_w, off_v, off_u, off_x, off_zc, off_tc, off_tf, off_s, off_bar, smem;
+    const __nv_bfloat16 *x;
+    int *status;
+    unsigned long long timeout_ns;
+    PrefetchList pf;
+};
+
+// Plans a call for the row-stream kernel on a GPU with num_sms SMs; returns
+// WL_ERR_UNSUPPORTED when it does not fit (M > 16, a rank above
+// kRowsMaxRank or not a multiple of 8, U / V not 16-byte aligned, more than
+// kRowsMaxBlocks blocks per CTA, or the shared-memory budget).
+wl_status plan_rows(RowsParams &p, int M, int K, const wl_proj *projs, int P, int num_sms);
+cudaError_t launch_rows(const RowsParams &p, cudaStream_t stream);
 
 // ----------------------------------------------------------------- GEMM ----
 // tcgen05 GEMM: Y[m][n] = s[n] * sum_k A[m][k] B[n][k] + sum_j T[m][j] U[n][j].
@@ -151,6 +217,7 @@ struct GemmParams {
     int num_tiles;
     int *status;
     unsigned long long timeout_ns;
+    PrefetchList pf;
 };
 
 void set_gemm_stages(GemmParams &p);
@@ -178,6 +245,11 @@ cudaError_t launch_pad_u(const __nv_bfloat16 *U, int N, int r, int r_pad,
 cudaError_t launch_materialize(const __nv_bfloat16 *W0, const float *s, const __nv_bfloat16 *U,
                                const __nv_bfloat16 *V, __nv_bfloat16 *Weff, int N, int K, int r,
                                cudaStream_t stream);
+
+// ----------------------------------------------------------- wait limit ----
+// Time limit of every device-side wait the forward kernels make (2 s unless
+// wl_set_wait_limit changed it).
+unsigned long long wait_limit_ns();
 
 // --------------------------------------------------------------- probes ----
 cudaError_t launch_wait_probe(int *flag, int *status, unsigned long long limit_ns,

@@ -28,6 +28,7 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB
 constexpr size_t kWordsBytes = 256;                // status word + arrival counters
+constexpr int kCounterWord = 8;                    // words [0, 8): status; [8, 64): counters
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -109,18 +110,36 @@ extern "C" wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *
     dp.a.K = K;
     dp.a.t_ld = r;
     dp.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-    dp.a.timeout_ns = 2000000000ull;
+    dp.a.timeout_ns = wait_limit_ns();
     DecodePlan plan;
     if ((st = plan_decode(dp, d->num_sms, &plan)) != WL_OK) return st;
     // Scratch: the word block, then the partial sums of V^T x ((grid+1) x M x r fp32).
     if (kWordsBytes + align256(plan.tpart_bytes) > kScratchBytes) return WL_ERR_UNSUPPORTED;
 
-    // The array keeps the previous call's contents: zero the status word and the
-    // arrival counters, which must start at zero, on the caller's stream.
-    if (cudaMemsetAsync(d->scratch, 0, kWordsBytes, stream) != cudaSuccess) return WL_ERR_CUDA;
+    // The array keeps the previous call's contents: zero the arrival counters,
+    // which must start at zero (a call whose wait gave up leaves them set), on
+    // the caller's stream.  The status word is kept until
+    // wl_noalloc_last_status() reads it.
     int *words = reinterpret_cast<int *>(d->scratch);
+    if (cudaMemsetAsync(words + kCounterWord, 0, kWordsBytes - kCounterWord * sizeof(int), stream) != cudaSuccess)
+        return WL_ERR_CUDA;
     dp.a.status = words;
-    dp.a.sync = reinterpret_cast<unsigned int *>(words + 8);
+    dp.a.sync = reinterpret_cast<unsigned int *>(words + kCounterWord);
     dp.a.Tpart = reinterpret_cast<float *>(d->scratch + kWordsBytes);
     return launch_decode(dp, plan, stream) == cudaSuccess ? WL_OK : WL_ERR_CUDA;
+}
+
+extern "C" wl_status wl_noalloc_last_status(void *stream) {
+    using namespace wl;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoAllocDevice *d = nullptr;
+    wl_status st = noalloc_setup(&d);
+    if (st != WL_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WL_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, d->scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WL_ERR_CUDA;
+    // after an error, clear the whole word block (status and any counters a
+    // call that gave up left set)
+    if (word != 0 && cudaMemset(d->scratch, 0, kWordsBytes) != cudaSuccess) return WL_ERR_CUDA;
+    return static_cast<wl_status>(word);
 }

@@ -33,8 +33,9 @@ def test_exports_every_declared_function(L):
 
 
 def test_status_strings(L):
-    for code in range(7):
+    for code in range(8):
         assert L.wl_status_string(code)
+    assert b"converge" in L.wl_status_string(7)
     assert L.wl_version() >= 1
 
 
@@ -95,3 +96,27 @@ def test_materialize_validation(L):
     # empty weights are a no-op and touch nothing
     assert mat(N=0, W0=None, s=None, U=None, V=None, out=None) == 0
     assert mat(K=0, W0=None, s=None, U=None, V=None, out=None) == 0
+
+
+def test_prefetch_validation(L):
+    """wl_stacked_forward_prefetch rejects bad range lists on the host, before
+    anything is launched."""
+    arr = (wl._Proj * 1)(wl._Proj(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 8))
+    rng = (wl._Range * (wl.MAX_PREFETCH + 1))()
+    fn = L.wl_stacked_forward_prefetch
+    assert fn(FAKE, 1, 16, arr, 1, 0, rng, -1, None) == 1
+    assert fn(FAKE, 1, 16, arr, 1, 0, rng, wl.MAX_PREFETCH + 1, None) == 1
+    assert fn(FAKE, 1, 16, arr, 1, 0, None, 1, None) == 1
+    rng[0] = wl._Range(None, 64)  # a NULL range with bytes
+    assert fn(FAKE, 1, 16, arr, 1, 0, rng, 1, None) == 1
+    # the call's own checks come first
+    assert fn(FAKE, 1, 12, arr, 1, 0, rng, 0, None) == 2
+    # empty calls are a no-op whatever the list holds
+    assert fn(FAKE, 0, 16, arr, 1, 0, rng, 0, None) == 0
+
+
+def test_wait_limit_validation(L):
+    assert L.wl_set_wait_limit(-1) == 1
+    assert L.wl_set_wait_limit(20_000_000_000) == 1
+    assert L.wl_set_wait_limit(1000) == 0
+    assert L.wl_set_wait_limit(0) == 0  # back to the default

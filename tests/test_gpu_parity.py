@@ -204,3 +204,29 @@ def test_stacked_fused_t_with_rank_zero_projection(M, ranks):
     assert plan["t_fused"] == 1
     call = wl_inputs.random_case(60 + M, M, [300, 200, 40][:len(ranks)], 520, ranks, P=len(ranks))
     check_call(call, "decode")
+
+
+# ------------------------------------------------------- L2 prefetch hint ---
+@pytest.mark.parametrize("path,M", [("decode", 1), ("decode", 8), ("gemm", 16), ("gemm", 130)])
+def test_prefetch_leaves_results_unchanged(path, M):
+    """wl_stacked_forward_prefetch only pulls ranges into L2: the outputs are
+    bit-identical to the call without it and match the oracle.  The ranges
+    include the next call's weights, an odd-sized range at an odd address, an
+    empty one, and the call's own output buffer."""
+    call = wl_inputs.random_case(31 + M, M, [700, 129], 1032, [16, 8], P=2)
+    nxt = wl_inputs.random_case(32 + M, 1, 2000, 1152, 16)
+    xd, pd = to_dev(call)
+    _, npd = to_dev(nxt)
+    base = wl.stacked_forward(xd, pd, path=path)
+    torch.cuda.synchronize()
+    ys = [torch.empty_like(y) for y in base]
+    odd = torch.empty(4099, dtype=torch.uint8, device="cuda")
+    pf = [t for t in npd[0]] + [(odd.data_ptr() + 3, 4093), (odd.data_ptr(), 0), ys[0]]
+    for _ in range(2):
+        wl.stacked_forward(xd, pd, ys=ys, path=path, prefetch=pf)
+    torch.cuda.synchronize()
+    assert wl.last_device_status() == 0
+    for p, y, yb in zip(call.projs, ys, base):
+        assert torch.equal(y, yb)
+        ref = oracle.forward(call.x, p.W0, p.s, p.U, p.V)
+        compare(y.double().cpu().numpy(), ref, f"prefetch {path} M={M}")
