@@ -6,22 +6,30 @@
 One step = one pass of the hot path over one batch of synthetic input.  The
 default workload is the Gemma-3-1B-shaped decode: 26 layers in 13 bands
 (G = 13), rank 16, M = 1 token, every layer's q/k/v (stacked), o, gate/up
-(stacked) and down projections.  The metric is weight GB/s: unique parameter
-bytes a step must stream (each band's W0 once, every layer's s, U, V) divided
-by the step time.  Inputs are resident in HBM before timing; per step they
-total more than 3x the 126 MB L2.
+(stacked) and down projections, each call naming the next calls' weights for
+the L2 prefetch (a decode step runs a fixed sequence of projections).  The
+metric is weight GB/s: unique parameter bytes a step must stream (each band's
+W0 once, every layer's s, U, V) divided by the step time.  Inputs are resident
+in HBM before timing; per step they total more than 3x the 126 MB L2.
 
 Timed region: CUDA-graph replays of the whole step (W >= 3 warm-up steps, then
 exactly K steps between two barrier + synchronize pairs, CUDA events on the
 launching stream, max over ranks).  The JSON line adds:
+  timing       the same graph replayed in windows for >= 1 s: median, p10,
+               p90 of the step time;
+  clocks       nvidia-smi samples every 10 ms over the timed region and that
+               window;
   e2e          the same metric through the public Python API, eager, with the
                step's x copied host->device from pinned memory and all y copied
                back every step;
   roofline     for the dominant kernel (the gate/up stacked decode call),
                timed alone over rotating buffers;
   cpu_baseline the fp64 oracle on the host, on a bounded sample of the step;
-  secondary    the other workloads' headline figures (Gemma-4-31B decode
-               GB/s, Gemma-4-31B prefill TFLOP/s).
+  secondary    every other workload's figures: the Gemma-3 dense comparator,
+               the Gemma-3 G=1 rank-64 stacks at M = 1, 8, 64, the Gemma-4-31B
+               decode families at M = 1 and 16, the Gemma-4-31B prefill
+               families (M = 4096), each a median over >= 1 s with p10 / p90
+               and its fraction of the measured peak.
 With --gpus N > 1 each rank runs an independent replica (the path has no
 exchange step); value is the total over ranks.
 """
@@ -29,9 +37,10 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import re
 import json
 import os
+import platform
+import re
 import statistics
 import subprocess
 import sys
@@ -48,6 +57,7 @@ from linear_wl_forward_b200 import footprint  # noqa: E402
 
 METRIC = "decode weight GB/s (% of HBM peak); prefill TFLOP/s (% bf16 TC peak)"
 L2_BYTES = 126 * 1024 * 1024
+PREFETCH_CALLS = 1  # calls ahead whose weights each call of the sweep prefetches into L2
 
 
 # ------------------------------------------------------------------ utils --
@@ -63,30 +73,47 @@ def load_peaks():
             "source": "fallback"}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons every 10 ms while active; the
+    samples carry host timestamps so a window can be cut out."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, period_ms=10):
         self.dev = device_index
+        self.period = period_ms
         self.proc = None
         self.out = None
+        self.t_start = None
 
     def __enter__(self):
         try:
             self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.t_start = time.time()
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.period)],
                 stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)  # nvidia-smi is sampling by the time the region starts
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.05)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -95,7 +122,7 @@ class ClockSampler:
 
     def summary(self):
         if self.proc is None or self.out is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.out.flush()
         with open(self.out.name) as f:
             rows = [[c.strip() for c in line.split(",")] for line in f if line.count(",") >= 8]
@@ -105,7 +132,8 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "period_ms": self.period}
 
 
 def to_dev_call(call):
@@ -114,69 +142,59 @@ def to_dev_call(call):
                        p.V.cuda() if p.r else None) for p in call.projs]}
 
 
-def launches_per_call(call, path):
-    """Kernels one call launches (the library's own kernels)."""
-    rs = [p.r for p in call.projs]
-    if path == "decode":
-        return 1  # one fused kernel: W0 x, V^T x and the epilogue
-    n = 1
-    if any(rs):
-        n += 2  # one V transpose for all projections + the T = x V GEMM
-        n += sum(1 for r in rs if r and r % 8)  # padded U copies
-    return n
-
-
-def call_path(call):
-    """The kernel path the library's automatic choice takes for a call (the
-    rule of wl_path in include/wl.h)."""
+def call_path(M, projs_nr, K=None):
+    """The kernel path the library's automatic choice takes for a call
+    (wl_path in include/wl.h): 'rows', 'decode' or 'gemm'."""
     import linear_wl_forward_b200 as wl
 
-    M = call.x.shape[0]
-    rows = sum(p.N for p in call.projs)
+    rows = sum(n for n, _ in projs_nr)
     if M <= 4 or (M <= wl.DECODE_MAX_M and rows < 8192):
+        if K is not None:
+            try:
+                wl.describe_rows_plan(M, K, projs_nr)
+                return "rows"
+            except wl.WLError:
+                pass
         return "decode"
     return "gemm"
 
 
-# ------------------------------------------------------------- workloads --
-def build_workload(name):
-    """Returns (calls, unique_weight_bytes, flops, description)."""
-    if name == "gemma3_decode":
-        calls = wl_inputs.gemma3_sweep(seed=2, G=13, r=16, M=1)
-        desc = {"workload": "Gemma-3-1B-shaped decode sweep", "layers": 26, "bands_G": 13,
-                "rank": 16, "M": 1, "hidden": 1152}
-    elif name == "gemma3_g1":
-        calls = wl_inputs.gemma3_sweep(seed=3, G=1, r=64, M=8)
-        desc = {"workload": "Gemma-3-1B-shaped stacked decode, G=1", "layers": 26, "rank": 64,
-                "M": 8}
-    elif name == "gemma4_decode":
-        calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=range(12))
-        desc = {"workload": "Gemma-4-31B-shaped decode, band 0 (layers 0-11)", "rank": 256,
-                "M": 1, "hidden": 5376}
-    elif name == "gemma4_prefill":
-        calls = wl_inputs.gemma4_calls(seed=5, r=256, M=4096, layers=[0])
-        desc = {"workload": "Gemma-4-31B-shaped prefill, sliding layer 0", "rank": 256,
-                "M": 4096, "hidden": 5376}
-    else:
-        raise SystemExit(f"unknown workload {name}")
-    seen = set()
-    wbytes = 0
-    flops = 0
-    for c in calls:
-        M = c.x.shape[0]
-        for p in c.projs:
-            if id(p.W0) not in seen:
-                seen.add(id(p.W0))
-                wbytes += p.N * p.K * 2
-            wbytes += (p.N + p.K) * p.r * 2 + p.N * 4
-            flops += footprint.call_flops(M, p.N, p.K, p.r)
-    return calls, wbytes, flops, desc
+def launches_per_call(path, ranks):
+    """Kernels one call launches (the library's own kernels)."""
+    if path in ("rows", "decode"):
+        return 1  # one fused kernel: W0 x, V^T x and the epilogue
+    n = 1
+    if any(ranks):
+        n += 2  # one V transpose for all projections + the T = x V GEMM
+        n += sum(1 for r in ranks if r and r % 8)  # padded U copies
+    return n
 
 
-def make_step(dev_calls, outs, wl):
+def prefetch_lists(dev_calls, ahead):
+    """For each call, the weights of the `ahead` calls after it (wrapping
+    around: the last calls of a step name the first ones of the next)."""
+    n = len(dev_calls)
+    out = []
+    for i in range(n):
+        items = []
+        for j in range(1, ahead + 1):
+            if j >= n:
+                break
+            for t in dev_calls[(i + j) % n]["projs"]:
+                items += [a for a in t if a is not None]
+        out.append(items)
+    return out
+
+
+def make_step(dev_calls, outs, wl, ahead=0):
+    """The step as prepared public-API calls (checks done once)."""
+    pfs = prefetch_lists(dev_calls, ahead)
+    prepared = [wl.prepare_stacked(dc["x"], dc["projs"], ys=ys, prefetch=pf)
+                for dc, ys, pf in zip(dev_calls, outs, pfs)]
+
     def step():
-        for dc, ys in zip(dev_calls, outs):
-            wl.stacked_forward(dc["x"], dc["projs"], ys=ys)
+        for p in prepared:
+            p()
     return step
 
 
@@ -223,6 +241,60 @@ def time_graph(g, reps):
     return start.elapsed_time(end) / reps  # ms
 
 
+def time_windows(g, seconds=1.0, min_windows=5):
+    """Graph replays in windows of about 50 ms until `seconds` have passed:
+    median, p10 and p90 of the per-replay time (ms) over the windows."""
+    one = time_graph(g, 3)
+    reps = max(1, int(0.05 / max(one * 1e-3, 1e-7)))
+    ts = []
+    t0 = time.perf_counter()
+    while len(ts) < min_windows or time.perf_counter() - t0 < seconds:
+        ts.append(time_graph(g, reps))
+    ts.sort()
+    q = lambda f: ts[min(len(ts) - 1, int(f * len(ts)))]  # noqa: E731
+    return {"median_ms": statistics.median(ts), "p10_ms": q(0.1), "p90_ms": q(0.9),
+            "windows": len(ts), "replays_per_window": reps, "seconds": round(time.perf_counter() - t0, 2)}
+
+
+def per_call(stats, n):
+    return {k: (v / n if k.endswith("_ms") else v) for k, v in stats.items()}
+
+
+# ------------------------------------------------------------- workloads --
+def build_workload(name):
+    """Returns (calls, unique_weight_bytes, flops, description)."""
+    if name == "gemma3_decode":
+        calls = wl_inputs.gemma3_sweep(seed=2, G=13, r=16, M=1)
+        desc = {"workload": "Gemma-3-1B-shaped decode sweep", "layers": 26, "bands_G": 13,
+                "rank": 16, "M": 1, "hidden": 1152}
+    elif name == "gemma3_g1":
+        calls = wl_inputs.gemma3_sweep(seed=3, G=1, r=64, M=8)
+        desc = {"workload": "Gemma-3-1B-shaped stacked decode, G=1", "layers": 26, "rank": 64,
+                "M": 8}
+    elif name == "gemma4_decode":
+        calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=range(12))
+        desc = {"workload": "Gemma-4-31B-shaped decode, band 0 (layers 0-11)", "rank": 256,
+                "M": 1, "hidden": 5376}
+    elif name == "gemma4_prefill":
+        calls = wl_inputs.gemma4_calls(seed=5, r=256, M=4096, layers=[0])
+        desc = {"workload": "Gemma-4-31B-shaped prefill, sliding layer 0", "rank": 256,
+                "M": 4096, "hidden": 5376}
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    seen = set()
+    wbytes = 0
+    flops = 0
+    for c in calls:
+        M = c.x.shape[0]
+        for p in c.projs:
+            if id(p.W0) not in seen:
+                seen.add(id(p.W0))
+                wbytes += p.N * p.K * 2
+            wbytes += (p.N + p.K) * p.r * 2 + p.N * 4
+            flops += footprint.call_flops(M, p.N, p.K, p.r)
+    return calls, wbytes, flops, desc
+
+
 # --------------------------------------------------------------- roofline --
 ROOFLINE_CALLS = {
     # name: (N per projection, K, r, M, label)
@@ -232,7 +304,7 @@ ROOFLINE_CALLS = {
 }
 
 
-def decode_roofline(wl, peaks, call="gemma3_gate_up"):
+def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     """One stacked decode call timed alone with CUDA events over a graph of
     calls that rotate through enough distinct bundles (> 3x L2) that every
     launch streams its weights from HBM.  The default is the dominant kernel
@@ -246,16 +318,19 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up"):
         calls.append(to_dev_call(c))
     outs = [[torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
             for _ in calls]
-    step = make_step(calls, outs, wl)
-    g = capture(step, 3)
-    ms = time_graph(g, 20) / copies
+    g = capture(make_step(calls, outs, wl), 3)
+    st = per_call(time_windows(g, seconds), copies)
+    ms = st["median_ms"]
     achieved = per_call / (ms * 1e-3) / 1e9
-    traffic = traffic_from_profile("decode_kernel", call)
-    return {"kernel": "decode_kernel (one launch per call: W0 x, V^T x and the epilogue fused)",
-            "call": label,
+    path = call_path(M, [(N, r), (N, r)], K)
+    kernel = {"rows": "rows_kernel", "decode": "decode_kernel"}.get(path, "gemm_kernel")
+    traffic = traffic_from_profile(kernel, call)
+    return {"kernel": f"{kernel} (one launch per call: W0 x, V^T x and the epilogue fused)",
+            "call": label, "path": path,
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic, "algorithmic_bytes": per_call, "us_per_launch": round(ms * 1e3, 3),
+            "us_p10": round(st["p10_ms"] * 1e3, 3), "us_p90": round(st["p90_ms"] * 1e3, 3),
             "peak_source": peaks["source"]}
 
 
@@ -284,31 +359,94 @@ def kernel_source_sha(path):
 
 
 # -------------------------------------------------------------- secondary --
-def secondary_figures(wl, peaks, headline_ms):
-    out = {"gemma3_decode_dense_comparator": dense_figure(wl, peaks, headline_ms)}
-    # Gemma-4-31B decode, M = 1: stacked gate/up of two bands (rotating, > L2)
-    calls = wl_inputs.gemma4_calls(seed=4, r=256, M=1, layers=[0, 12], families=("gate",))
-    dev = [to_dev_call(c) for c in calls]
-    outs, _ = alloc_outputs(calls)
-    g = capture(make_step(dev, outs, wl), 3)
-    ms = time_graph(g, 10) / len(calls)
-    p0 = calls[0].projs
-    b = sum(footprint.call_weight_bytes(p.N, p.K, p.r) for p in p0)
-    out["gemma4_decode_gate_up_M1"] = {
-        "GB/s": round(b / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-        "us_per_call": round(ms * 1e3, 2), "weight_bytes_per_call": b}
-    del dev, outs, g
-    torch.cuda.empty_cache()
-    out.update(gemma4_layer_figures(wl, peaks))
-    out["gemma4_prefill_gate_up_M4096"] = prefill_figure(wl, peaks)
+def _figure(stats, n_calls, work, kind, peaks, extra=None):
+    """One secondary figure: `work` bytes (kind 'GB/s') or flops ('TFLOP/s')
+    per call, times per call from the windows' median, p10, p90."""
+    s = per_call(stats, n_calls)
+    ms = s["median_ms"]
+    if kind == "GB/s":
+        v = work / (ms * 1e-3) / 1e9
+        fr = v / peaks["hbm_gbs"]
+    else:
+        v = work / (ms * 1e-3) / 1e12
+        fr = v / peaks["bf16_tflops"]
+    out = {kind: round(v, 1), ("hbm_frac" if kind == "GB/s" else "tc_frac"): round(fr, 4),
+           "us_per_call": round(ms * 1e3, 2), "us_p10": round(s["p10_ms"] * 1e3, 2),
+           "us_p90": round(s["p90_ms"] * 1e3, 2), "windows": s["windows"]}
+    if extra:
+        out.update(extra)
     return out
 
 
-def dense_figure(wl, peaks, headline_ms):
+def rotating_figure(wl, peaks, stacks, M, K, copies, seconds, key, kind="GB/s", ahead=0):
+    """Calls of one stack shape [(N, r), ...] over `copies` distinct bundles
+    drawn on the device, replayed in a graph; work per call is the stack's
+    weight bytes (GB/s) or flops (TFLOP/s)."""
+    x = wl_inputs.device_x(M, K, key, M)
+    dev = []
+    for c in range(copies):
+        projs = [wl_inputs.device_bundle(N, K, r, key, c, i) for i, (N, r) in enumerate(stacks)]
+        dev.append({"x": x, "projs": projs})
+    outs = [[torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for N, _ in stacks] for _ in dev]
+    g = capture(make_step(dev, outs, wl, ahead), 3)
+    stats = time_windows(g, seconds)
+    assert wl.last_device_status() == 0
+    path = call_path(M, stacks, K)
+    if kind == "GB/s":
+        work = sum(footprint.call_weight_bytes(N, K, r) for N, r in stacks)
+    else:
+        work = sum(footprint.call_flops(M, N, K, r) for N, r in stacks)
+    fig = _figure(stats, copies, work, kind, peaks,
+                  {"path": path, "copies": copies, ("weight_bytes_per_call" if kind == "GB/s" else
+                                                    "flops_per_call"): work})
+    del g, dev, outs
+    torch.cuda.empty_cache()
+    return fig
+
+
+def secondary_figures(wl, peaks, headline_ms, seconds):
+    out = {"gemma3_decode_dense_comparator": dense_figure(wl, peaks, headline_ms, seconds)}
+    # Gemma-3-1B G = 1, rank 64: the stacked q/k/v and gate/up calls at 1, 8
+    # and 64 tokens over >= 12 bundle copies (> 400 MB, L2 defeated)
+    for name, stacks in (("qkv", [(1024, 64), (256, 64), (256, 64)]), ("gate_up", [(4096, 64), (4096, 64)])):
+        K = 1152
+        stack_bytes = sum(N * K * 2 for N, _ in stacks)
+        copies = max(12, (3 * L2_BYTES) // stack_bytes + 1)
+        for M in (1, 8, 64):
+            out[f"gemma3_g1_r64_{name}_M{M}"] = rotating_figure(
+                wl, peaks, stacks, M, K, copies, seconds, ("g3g1", name, M))
+    # Gemma-4-31B decode, rank 256, each stack family at M = 1 and 16 over
+    # three distinct bundles (every call streams from HBM)
+    g4 = {"qkv_sliding": ([(8192, 256), (4096, 256), (4096, 256)], 5376),
+          "o_sliding": ([(5376, 256)], 8192),
+          "qk_full": ([(16384, 256), (2048, 256)], 5376),
+          "o_full": ([(5376, 256)], 16384),
+          "gate_up": ([(21504, 256), (21504, 256)], 5376),
+          "down": ([(5376, 256)], 21504)}
+    for M in (1, 16):
+        for name, (stacks, K) in g4.items():
+            out[f"gemma4_decode_{name}_M{M}"] = rotating_figure(
+                wl, peaks, stacks, M, K, 3, seconds, ("g4d", name, M))
+    out.update(gemma4_layer_figures(wl, peaks, seconds))
+    # Gemma-4-31B prefill, M = 4096: every family and the stacks
+    g5 = {"q_sliding": ([(8192, 256)], 5376), "kv_sliding": ([(4096, 256)], 5376),
+          "q_full": ([(16384, 256)], 5376), "k_full": ([(2048, 256)], 5376),
+          "o_sliding": ([(5376, 256)], 8192), "o_full": ([(5376, 256)], 16384),
+          "gate_up": ([(21504, 256), (21504, 256)], 5376), "down": ([(5376, 256)], 21504),
+          "qkv_sliding_stacked": ([(8192, 256), (4096, 256), (4096, 256)], 5376),
+          "qk_full_stacked": ([(16384, 256), (2048, 256)], 5376)}
+    for name, (stacks, K) in g5.items():
+        out[f"gemma4_prefill_{name}_M4096"] = rotating_figure(
+            wl, peaks, stacks, 4096, K, 1, seconds, ("g4p", name), kind="TFLOP/s")
+    return out
+
+
+def dense_figure(wl, peaks, headline_ms, seconds):
     """The dense comparator of the Gemma-3-1B decode sweep: every projection's
     W_eff = diag(s) W0 + U V^T rebuilt once on the GPU (wl.materialize_weight),
     then the same 26-layer sweep as a plain rank-0 forward over the 26 distinct
-    dense weights.  Reported against the weightless sweep's time per step."""
+    dense weights, with the same cross-call prefetch.  Reported against the
+    weightless sweep's time per step."""
     calls = wl_inputs.gemma3_sweep(seed=2, G=13, r=16, M=1)
     dev = []
     wbytes = 0
@@ -324,17 +462,18 @@ def dense_figure(wl, peaks, headline_ms):
     torch.cuda.synchronize()
     assert wl.last_device_status() == 0
     outs, _ = alloc_outputs(calls)
-    g = capture(make_step(dev, outs, wl), 3)
-    ms = time_graph(g, 50)
+    g = capture(make_step(dev, outs, wl, PREFETCH_CALLS), 3)
+    st = time_windows(g, seconds)
+    ms = st["median_ms"]
     del dev, outs, g
     torch.cuda.empty_cache()
     gbs = wbytes / (ms * 1e-3) / 1e9
-    return {"ms_per_step": round(ms, 4), "GB/s": round(gbs, 1),
-            "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "weight_bytes_per_step": wbytes,
-            "weightless_over_dense_time": round(headline_ms / ms, 4)}
+    return {"ms_per_step": round(ms, 4), "p10_ms": round(st["p10_ms"], 4), "p90_ms": round(st["p90_ms"], 4),
+            "GB/s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+            "weight_bytes_per_step": wbytes, "weightless_over_dense_time": round(headline_ms / ms, 4)}
 
 
-def gemma4_layer_figures(wl, peaks):
+def gemma4_layer_figures(wl, peaks, seconds):
     """A whole Gemma-4-31B sliding layer (q/k/v stack, o, gate/up stack, down;
     rank 256) at M = 1 and M = 16 through the library's automatic path choice:
     two layers of different bands (distinct W0, > L2) in one graph, reported
@@ -354,32 +493,27 @@ def gemma4_layer_figures(wl, peaks):
             dev_m.append({"x": xs[K], "projs": dc["projs"]})
             calls_m.append(wl_inputs.Call(c.layer, c.projs, xs[K]))
         outs, _ = alloc_outputs(calls_m)
-        g = capture(make_step(dev_m, outs, wl), 3)
-        ms = time_graph(g, 5) / 2
+        g = capture(make_step(dev_m, outs, wl, PREFETCH_CALLS), 3)
+        st = per_call(time_windows(g, seconds), 2)
+        ms = st["median_ms"]
         gbs = wbytes / (ms * 1e-3) / 1e9
         out[f"gemma4_decode_sliding_layer_M{M}"] = {
             "GB/s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
-            "us_per_layer": round(ms * 1e3, 1), "weight_bytes_per_layer": wbytes,
-            "paths": [call_path(c) for c in calls_m if c.layer == 0]}
+            "us_per_layer": round(ms * 1e3, 1), "us_p10": round(st["p10_ms"] * 1e3, 1),
+            "us_p90": round(st["p90_ms"] * 1e3, 1), "weight_bytes_per_layer": wbytes,
+            "paths": [call_path(M, [(p.N, p.r) for p in c.projs], c.x.shape[1])
+                      for c in calls_m if c.layer == 0]}
         del outs, g
     del dev
     torch.cuda.empty_cache()
     return out
 
 
-def prefill_figure(wl, peaks):
+def prefill_figure(wl, peaks, seconds=1.0):
     """Gemma-4-31B prefill, M = 4096: the stacked gate/up call of layer 0
     (2 x 21504 x 5376, rank 256) on the tensor-core path."""
-    calls = wl_inputs.gemma4_calls(seed=5, r=256, M=4096, layers=[0], families=("gate",))
-    dev = [to_dev_call(c) for c in calls]
-    outs, _ = alloc_outputs(calls)
-    g = capture(make_step(dev, outs, wl), 3)
-    ms = time_graph(g, 5)
-    c = calls[0]
-    fl = sum(footprint.call_flops(4096, p.N, p.K, p.r) for p in c.projs)
-    tf = fl / (ms * 1e-3) / 1e12
-    return {"TFLOP/s": round(tf, 1), "tc_frac": round(tf / peaks["bf16_tflops"], 4),
-            "ms_per_call": round(ms, 3), "flops_per_call": fl, "peak": peaks["bf16_tflops"]}
+    return rotating_figure(wl, peaks, [(21504, 256), (21504, 256)], 4096, 5376, 1, seconds,
+                           ("g4p", "gate_up"), kind="TFLOP/s")
 
 
 # ---------------------------------------------------------- CPU baseline --
@@ -403,6 +537,11 @@ def oracle_sample(calls, budget_s=12.0):
         if time.perf_counter() - t0 > budget_s:
             break
     return done_b, time.perf_counter() - t0, n
+
+
+def cpu_baseline_line(value, sample):
+    return {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+            "host_cpu_count": os.cpu_count(), "cpu_model": cpu_model()}
 
 
 # ------------------------------------------------------------------- main --
@@ -451,8 +590,7 @@ def run_reference(args):
             "ms_per_step": round(s / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(desc, sample="oracle over whole calls of the step, bounded by time"),
-            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{sum(x[2] for x in samples)} calls over {args.steps} steps"},
+            "cpu_baseline": cpu_baseline_line(v, f"{sum(x[2] for x in samples)} calls over {args.steps} steps"),
             "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -465,6 +603,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gemma3_decode")
+    ap.add_argument("--prefetch", type=int, default=PREFETCH_CALLS,
+                    help="calls ahead whose weights each call prefetches into L2 (0: none)")
+    ap.add_argument("--seconds", type=float, default=1.0, help="time per figure's repeat windows")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--roofline-only", action="store_true",
                     help="time only the dominant kernel's call (the command the ncu summaries profile)")
@@ -495,10 +636,10 @@ def main():
     wl.lib()  # fails loudly if the CUDA library is missing
     peaks = load_peaks()
     if args.roofline_only:
-        print(json.dumps({"roofline": decode_roofline(wl, peaks, args.call)}), flush=True)
+        print(json.dumps({"roofline": decode_roofline(wl, peaks, args.call, args.seconds)}), flush=True)
         return
     if args.prefill_only:
-        print(json.dumps({"prefill": prefill_figure(wl, peaks)}), flush=True)
+        print(json.dumps({"prefill": prefill_figure(wl, peaks, args.seconds)}), flush=True)
         return
 
     calls, wbytes, flops, desc = build_workload(args.workload)
@@ -506,8 +647,9 @@ def main():
     total_out = sum(c.x.shape[0] * p.N for c in calls for p in c.projs)
     out_flat = torch.empty(total_out, dtype=torch.bfloat16, device="cuda")
     outs, _ = alloc_outputs(calls, out_flat)
-    step = make_step(dev_calls, outs, wl)
-    launches = sum(launches_per_call(c, call_path(c)) for c in calls)
+    step = make_step(dev_calls, outs, wl, args.prefetch)
+    paths = [call_path(c.x.shape[0], [(p.N, p.r) for p in c.projs], c.x.shape[1]) for c in calls]
+    launches = sum(launches_per_call(pth, [p.r for p in c.projs]) for c, pth in zip(calls, paths))
 
     graph = capture(step, args.warmup)
     for _ in range(args.warmup):
@@ -524,8 +666,10 @@ def main():
             graph.replay()
         end.record()
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+        if world > 1:
+            torch.distributed.barrier()
+        # the same graph in windows for >= 1 s (every rank, same collective steps)
+        windows = time_windows(graph, args.seconds)
     ms_total = max_over_ranks(start.elapsed_time(end), world, "cuda")
     status = wl.last_device_status()
     ms_step = ms_total / args.steps
@@ -543,14 +687,10 @@ def main():
     d2h = total_out * 2
     e2e_steps = max(3, min(args.steps, 10))
 
-    # the public API a decode loop uses: each call prepared once, issued per step
-    prepared = [wl.prepare_stacked(dc["x"], dc["projs"], ys=ys) for dc, ys in zip(dev_calls, outs)]
-
     def e2e_step():
         for k, t in xs_host.items():
             x_dev[k].copy_(t, non_blocking=True)
-        for call in prepared:
-            call()
+        step()  # the prepared public-API calls
         y_host.copy_(out_flat, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
@@ -575,11 +715,13 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 bundles, U(0.9,1.1) fp32 s, N(0,1) bf16 x)",
         "config": dict(desc, parallelism=f"replicas{world}" if world > 1 else "single GPU",
-                       unique_weight_bytes_per_step=wbytes,
+                       unique_weight_bytes_per_step=wbytes, prefetch_calls_ahead=args.prefetch,
+                       paths={p: paths.count(p) for p in sorted(set(paths))},
                        l2="inputs larger than L2: each step streams %.0f MB of unique weights"
                           % (wbytes / 1e6),
                        timing="CUDA graph of the whole step, replayed K times"),
         "hbm_frac": round(value / world / peaks["hbm_gbs"], 4),
+        "timing": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in windows.items()},
         "peaks": peaks,
         "gpu_launches": launches * args.steps,
         "device_status": wl.STATUS.get(status, status),
@@ -590,14 +732,14 @@ def main():
                        "one call per projection stack per step), x H2D (pinned) and all y D2H"},
     }
     if rank == 0 and world == 1:
-        line["roofline"] = decode_roofline(wl, peaks)
-        if not args.no_secondary:
-            line["secondary"] = secondary_figures(wl, peaks, ms_step)
+        with ClockSampler(local) as clk2:
+            line["roofline"] = decode_roofline(wl, peaks, seconds=args.seconds)
+            if not args.no_secondary:
+                line["secondary"] = secondary_figures(wl, peaks, ms_step, args.seconds)
+        line["secondary_clocks"] = clk2.summary()
         b, s, n = oracle_sample(calls, budget_s=12.0)
-        line["cpu_baseline"] = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": 1,
-                                "kind": "oracle",
-                                "sample": f"first {n} of {len(calls)} calls of one step "
-                                          f"({b / 1e6:.0f} MB of weights, {s:.1f} s)"}
+        line["cpu_baseline"] = cpu_baseline_line(
+            b / s / 1e9, f"first {n} of {len(calls)} calls of one step ({b / 1e6:.0f} MB of weights, {s:.1f} s)")
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -41,7 +41,7 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
-                        uint32_t box_cols, uint32_t box_rows) {
+                        uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return WL_ERR_CUDA;
     const cuuint64_t dims[2] = {cols, rows};
@@ -49,7 +49,8 @@ wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
-                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
 }
@@ -663,8 +664,9 @@ wl_status wl_describe_rows_plan(int M, int K, const wl_proj *projs, int P, int n
     alignas(16) static const unsigned char no_x[16] = {};
     wl_status st = wl::validate(reinterpret_cast<const wl_bf16 *>(no_x), M, K, projs, P, WL_PATH_ROWS);
     if (st != WL_OK) return st;
-    wl::RowsParams rp;
-    if ((st = wl::plan_rows(rp, M, K, projs, P, num_sms)) != WL_OK) return st;
+    static wl::RowsParams rp;  // large (tensor maps); guarded by g_mu
+    std::lock_guard<std::mutex> lock(wl::g_mu);
+    if ((st = wl::plan_rows(rp, M, K, projs, P, num_sms, false)) != WL_OK) return st;
     out->grid = rp.ngroups * rp.c;
     out->cluster = rp.c;
     out->row_groups = rp.ngroups;

@@ -62,15 +62,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete, giving up
-// after `limit_ns`.  On time-out records WL_ERR_TIMEOUT and returns false.
+// after `limit_ns` (the clock is read after every unsuccessful try, each of
+// which may itself suspend the thread for a while).  On time-out records
+// WL_ERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status,
                                           uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t polls = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((++polls & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             record_status(status, kStatusTimeout);
             return false;
         }

@@ -95,9 +95,8 @@ __device__ __forceinline__ void red_release_gpu_add(unsigned int *p, unsigned in
 // Wait (bounded) until a grid-wide counter reaches `expected`.
 __device__ __forceinline__ bool grid_wait(const unsigned int *ctr, unsigned int expected, const DecodeArgs &p) {
     const uint64_t t0 = globaltimer_ns();
-    uint32_t polls = 0;
     while (ld_acquire_gpu(ctr) < expected) {
-        if ((++polls & 63u) == 0 && globaltimer_ns() - t0 > p.timeout_ns) {
+        if (globaltimer_ns() - t0 > p.timeout_ns) {
             record_status(p.status, kStatusTimeout);
             return false;
         }

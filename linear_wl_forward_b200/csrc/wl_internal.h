@@ -119,9 +119,10 @@ struct DecodePlan {
 wl_status plan_decode(DecodeParams &p, int num_sms, DecodePlan *plan, bool encode_maps = true);
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
 
-// 2-D / 3-D bf16 tensor maps with 128-byte swizzling; out-of-range reads give 0.
+// 2-D / 3-D bf16 tensor maps (128-byte swizzling unless swizzle128 is false);
+// out-of-range reads give 0.
 wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
-                        uint32_t box_cols, uint32_t box_rows);
+                        uint32_t box_cols, uint32_t box_rows, bool swizzle128 = true);
 wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                         uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
                         uint32_t b2);
@@ -130,9 +131,10 @@ wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d
 // Row-stream decode kernel for short calls (latency-bound: a few MB of
 // weights).  Each CTA owns a group of up to kRowsMaxBlocks 16-row blocks of
 // one projection and, with a cluster of c CTAs, 1/c of K; before the wait for
-// the previous kernel its lanes copy their W0 MMA fragments into shared
-// memory (cp.async) and V and U rows are bulk-copied there, and the partial
-// sums of the c CTAs meet over distributed shared memory.
+// the previous kernel its warps copy their share of W0 into shared memory
+// (TMA tiles laid out as the lanes' MMA fragments) and V and U rows are
+// bulk-copied there, and the partial sums of the c CTAs meet over
+// distributed shared memory.
 constexpr int kRowsWarps = 8;
 constexpr int kRowsThreads = 32 * kRowsWarps;
 constexpr int kRowsKGroup = 32;     // K columns per warp step (two m16n8k16 MMAs)
@@ -153,6 +155,7 @@ struct RowsSeg {
 };
 
 struct RowsParams {
+    CUtensorMap tm_w[kMaxSeg];  // W0_p: 2-D {K, N_p}, box {32, 16 nb_p}, no swizzle
     RowsSeg seg[kMaxSeg];
     int nseg;
     int M, K;
@@ -172,8 +175,10 @@ struct RowsParams {
 // Plans a call for the row-stream kernel on a GPU with num_sms SMs; returns
 // WL_ERR_UNSUPPORTED when it does not fit (M > 16, a rank above
 // kRowsMaxRank or not a multiple of 8, U / V not 16-byte aligned, more than
-// kRowsMaxBlocks blocks per CTA, or the shared-memory budget).
-wl_status plan_rows(RowsParams &p, int M, int K, const wl_proj *projs, int P, int num_sms);
+// kRowsMaxBlocks blocks per CTA, or the shared-memory budget).  encode_maps =
+// false plans without the tensor maps (host logic only).
+wl_status plan_rows(RowsParams &p, int M, int K, const wl_proj *projs, int P, int num_sms,
+                    bool encode_maps = true);
 cudaError_t launch_rows(const RowsParams &p, cudaStream_t stream);
 
 // ----------------------------------------------------------------- GEMM ----

@@ -38,7 +38,7 @@ def test_rows_clusters_of_each_size():
     """The planner's cluster sizes 1, 2 and 4 all occur among these calls and
     each matches the oracle."""
     seen = set()
-    for M, N, K, r in [(1, 6000, 1152, 16), (1, 3000, 1152, 16), (2, 600, 2048, 16), (1, 1152, 4096, 16)]:
+    for M, N, K, r in [(1, 6000, 1152, 16), (1, 3000, 1152, 16), (2, 600, 2048, 16), (1, 600, 8192, 16)]:
         seen.add(wl.describe_rows_plan(M, K, [(N, r)])["cluster"])
         check_call(wl_inputs.random_case(90 + N, M, N, K, r), "rows")
     assert seen == {1, 2, 4}, seen
@@ -64,36 +64,41 @@ def test_rows_gemma3_1b_layer(M):
         try:
             wl.describe_rows_plan(M, call.projs[0].K, shapes)
         except wl.WLError:
-            # 16 tokens of the 8192-row gate/up stack need more shared memory
+            # 8 or 16 tokens of the 8192-row gate/up stack need more shared memory
             # than two CTAs per SM allow: that call takes another kernel
-            assert M == 16 and [p.family for p in call.projs] == ["gate", "up"]
+            assert M >= 8 and [p.family for p in call.projs] == ["gate", "up"]
             continue
         check_call(call, "rows")
 
 
-def test_rows_deterministic_and_matches_decode_kernel_bits_on_integers():
-    """Repeat calls give identical bits; on small integers (exact in bf16 and
-    fp32) the row-stream kernel equals the oracle bit for bit."""
+def test_rows_deterministic():
+    """Repeat calls give identical bits."""
     call = wl_inputs.random_case(8, 4, 700, 1544, 64)
     xd, pd = to_dev(call)
     a = run(call, "rows", xd, pd)[0]
     b = run(call, "rows", xd, pd)[0]
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("M,N,K,r,x_zero,cluster", [(5, 200, 1000, 16, 0.6, 1), (2, 600, 8192, 16, 0.95, 4),
+                                                   (3, 300, 8192, 24, 0.95, 4)])
+def test_rows_bit_exact_on_small_integers(M, N, K, r, x_zero, cluster):
+    """Inputs in {-1, 0, 1} (x sparse enough that every sum stays small) and
+    half-integer scales: every partial sum is exact in fp32 and every y is a
+    bf16 value, so the kernel -- without clusters and with the cluster's
+    sums over distributed shared memory -- must equal the oracle bit for bit."""
+    assert wl.describe_rows_plan(M, K, [(N, r)])["cluster"] == cluster
     rng = np.random.default_rng(4)
-    M, N, K, r = 5, 200, 1000, 16
 
     def draw(shape, p0):  # -1, 0, 1 with P(0) = p0
         return torch.tensor(rng.choice([-1, 0, 1], size=shape, p=[(1 - p0) / 2, p0, (1 - p0) / 2]),
                             dtype=torch.bfloat16)
 
-    x, W0, U, V = draw((M, K), 0.6), draw((N, K), 0.6), draw((N, r), 0.5), draw((K, r), 0.6)
+    x, W0, U, V = draw((M, K), x_zero), draw((N, K), 0.6), draw((N, r), 0.5), draw((K, r), 0.6)
     s = torch.tensor(rng.integers(-2, 3, (N,)) * 0.5, dtype=torch.float32)
     ref = oracle.forward(x, W0, s, U, V)
-    # every partial sum is a small half-integer (exact in fp32) and so is y;
-    # each y is a bf16 value, so a correct kernel rounds nothing
     assert np.all(ref == np.round(ref * 2) / 2) and np.max(np.abs(ref)) < 2 ** 20
     assert np.array_equal(torch.tensor(ref).to(torch.bfloat16).double().numpy(), ref)
-    assert wl.describe_rows_plan(M, K, [(N, r)])["cluster"] == 4
     y = wl.stacked_forward(x.cuda(), [(W0.cuda(), s.cuda(), U.cuda(), V.cuda())], path="rows")[0]
     assert np.array_equal(y.float().cpu().numpy(), ref)
 

@@ -271,3 +271,25 @@ def random_case(seed: int, M: int, N: int, K: int, r: int, P: int = 1):
         projs.append(Proj(f"f{p}", W0, s, U, V))
     x = draw_x(wl, seed, M, K)
     return Call(0, projs, x)
+
+
+# ------------------------------------------------------- device draws -------
+def device_bundle(N: int, K: int, r: int, *key, device="cuda"):
+    """(W0, s, U, V) drawn directly on `device` with the distributions above
+    (W0, U, V ~ N(0, 0.02) bf16, s ~ U(0.9, 1.1) fp32) from a generator seeded
+    by the key: for timing runs, where drawing hundreds of MB on the CPU would
+    dominate.  A different random stream from the CPU draws."""
+    g = torch.Generator(device=device)
+    g.manual_seed(subseed("device", *key))
+    W0 = (torch.randn(N, K, generator=g, device=device) * W_STD).to(torch.bfloat16)
+    s = torch.rand(N, generator=g, device=device) * (S_HI - S_LO) + S_LO
+    U = (torch.randn(N, r, generator=g, device=device) * W_STD).to(torch.bfloat16) if r else None
+    V = (torch.randn(K, r, generator=g, device=device) * W_STD).to(torch.bfloat16) if r else None
+    return W0, s, U, V
+
+
+def device_x(M: int, K: int, *key, device="cuda"):
+    """x ~ N(0, 1) bf16 drawn on `device` (see device_bundle)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(subseed("device-x", *key))
+    return torch.randn(M, K, generator=g, device=device).to(torch.bfloat16)
