@@ -6,9 +6,9 @@
 One step = one pass of the hot path over one batch of synthetic input.  The
 default workload is the Gemma-3-1B-shaped decode: 26 layers in 13 bands
 (G = 13), rank 16, M = 1 token, every layer's q/k/v (stacked), o, gate/up
-(stacked) and down projections, each call naming the next calls' weights for
-the L2 prefetch (a decode step runs a fixed sequence of projections).  The
-metric is weight GB/s: unique parameter bytes a step must stream (each band's
+(stacked) and down projections (--prefetch N: each call also names the next
+N calls' weights for the L2 prefetch; 0 by default, which measured fastest).
+The metric is weight GB/s: unique parameter bytes a step must stream (each band's
 W0 once, every layer's s, U, V) divided by the step time.  Inputs are resident
 in HBM before timing; per step they total more than 3x the 126 MB L2.
 
@@ -57,7 +57,7 @@ from linear_wl_forward_b200 import footprint  # noqa: E402
 
 METRIC = "decode weight GB/s (% of HBM peak); prefill TFLOP/s (% bf16 TC peak)"
 L2_BYTES = 126 * 1024 * 1024
-PREFETCH_CALLS = 1  # calls ahead whose weights each call of the sweep prefetches into L2
+PREFETCH_CALLS = 0  # calls ahead whose weights each call of the sweep prefetches into L2 (measured: none is fastest)
 
 
 # ------------------------------------------------------------------ utils --

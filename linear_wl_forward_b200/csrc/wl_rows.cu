@@ -218,8 +218,6 @@ __global__ void __launch_bounds__(RTH, 2) rows_kernel(const __grid_constant__ Ro
         for (int kl = 0; kl < nkw; ++kl)
             tma_tile_2d(wbase + (size_t)kl * bb * 1024u, &P.tm_w[sp], k0 + (kgA + kl) * KG, row0, &wbar[warp], pol);
     }
-    // the following call's weights into L2
-    if (tid == 32) l2_prefetch_share(P.pf, blockIdx.x, gridDim.x);
     // The outputs this CTA writes: rows [er0, er1) of the group, every token;
     // their scales into shared memory (the barrier below keeps these loads
     // ahead of the wait for the previous kernel).
@@ -232,6 +230,9 @@ __global__ void __launch_bounds__(RTH, 2) rows_kernel(const __grid_constant__ Ro
     bool ok = true;
     if (r > 0) ok = mbar_wait(bar, 0, P.status, P.timeout_ns);
     if (nkw > 0 && !mbar_wait(&wbar[warp], 0, P.status, P.timeout_ns)) ok = false;
+    // The following call's weights into L2, once this warp's own copies have
+    // landed (the prefetches take the same copy engine).
+    if (warp == RW - 1 && lane == 0) l2_prefetch_share(P.pf, blockIdx.x, gridDim.x);
 
     pdl_wait_primary();  // the previous kernel is done: x is ready, y is ours
     // x: each warp stages the columns of its own k-groups (no CTA barrier),
