@@ -19,9 +19,10 @@ launching stream, max over ranks).  The JSON line adds:
                p90 of the step time;
   clocks       nvidia-smi samples every 10 ms over the timed region and that
                window;
-  e2e          the same metric through the public Python API, eager, with the
-               step's x copied host->device from pinned memory and all y copied
-               back every step;
+  e2e          the same metric through the public API (the step's calls
+               captured once into a CUDA graph), with the step's x copied
+               host->device from pinned memory and all y copied back every
+               step; eager_value issues the same calls from Python instead;
   roofline     for the dominant kernel (the gate/up stacked decode call),
                timed alone over rotating buffers;
   cpu_baseline the fp64 oracle on the host, on a bounded sample of the step;
@@ -310,7 +311,7 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     launch streams its weights from HBM.  The default is the dominant kernel
     of the Gemma-3-1B decode step: the stacked gate/up call."""
     N, K, r, M, label = ROOFLINE_CALLS[call]
-    per_call = 2 * footprint.call_weight_bytes(N, K, r) + footprint.call_io_bytes(M, 2 * N, K)
+    call_bytes = 2 * footprint.call_weight_bytes(N, K, r) + footprint.call_io_bytes(M, 2 * N, K)
     copies = max(4, (3 * L2_BYTES) // (2 * N * K * 2) + 1)
     calls = []
     for i in range(copies):
@@ -321,7 +322,7 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     g = capture(make_step(calls, outs, wl), 3)
     st = per_call(time_windows(g, seconds), copies)
     ms = st["median_ms"]
-    achieved = per_call / (ms * 1e-3) / 1e9
+    achieved = call_bytes / (ms * 1e-3) / 1e9
     path = call_path(M, [(N, r), (N, r)], K)
     kernel = {"rows": "rows_kernel", "decode": "decode_kernel"}.get(path, "gemm_kernel")
     traffic = traffic_from_profile(kernel, call)
@@ -329,7 +330,7 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
             "call": label, "path": path,
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic, "algorithmic_bytes": per_call, "us_per_launch": round(ms * 1e3, 3),
+            "traffic": traffic, "algorithmic_bytes": call_bytes, "us_per_launch": round(ms * 1e3, 3),
             "us_p10": round(st["p10_ms"] * 1e3, 3), "us_p90": round(st["p90_ms"] * 1e3, 3),
             "peak_source": peaks["source"]}
 
@@ -687,26 +688,32 @@ def main():
     d2h = total_out * 2
     e2e_steps = max(3, min(args.steps, 10))
 
-    def e2e_step():
-        for k, t in xs_host.items():
-            x_dev[k].copy_(t, non_blocking=True)
-        step()  # the prepared public-API calls
-        y_host.copy_(out_flat, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+    def e2e_run(issue):
+        def one():
+            for k, t in xs_host.items():
+                x_dev[k].copy_(t, non_blocking=True)
+            issue()
+            y_host.copy_(out_flat, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
 
-    for _ in range(2):
-        e2e_step()
-    if world > 1:
-        torch.distributed.barrier()
-    t0 = time.perf_counter()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3) / e2e_steps,
-                            world, "cuda")
+        for _ in range(2):
+            one()
+        if world > 1:
+            torch.distributed.barrier()
+        t0 = time.perf_counter()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            one()
+        e1.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3) / e2e_steps,
+                              world, "cuda")
+
+    # the step's public-API calls captured once into a CUDA graph, as a decode
+    # loop issues them; and the same calls issued eagerly from Python
+    e2e_ms = e2e_run(graph.replay)
+    e2e_eager_ms = e2e_run(step)
     e2e_value = replica_value(world, wbytes, 1, e2e_ms)
 
     line = {
@@ -728,8 +735,11 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
-                "how": "eager calls of the public API (wl.prepare_stacked once per call, then "
-                       "one call per projection stack per step), x H2D (pinned) and all y D2H"},
+                "how": "public-API calls (wl.prepare_stacked once per projection stack) captured "
+                       "once into a CUDA graph and replayed per step, with x copied H2D from pinned "
+                       "memory before and every y copied D2H after, inside the timed region",
+                "eager_value": round(replica_value(world, wbytes, 1, e2e_eager_ms), 2),
+                "eager_ms_per_step": round(e2e_eager_ms, 3)},
     }
     if rank == 0 and world == 1:
         with ClockSampler(local) as clk2:
