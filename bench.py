@@ -23,12 +23,15 @@ launching stream, max over ranks).  The JSON line adds:
                captured once into a CUDA graph), with the step's x copied
                host->device from pinned memory and all y copied back every
                step; eager_value issues the same calls from Python instead;
-  roofline     for the dominant kernel (the gate/up stacked decode call),
-               timed alone over rotating buffers;
+  roofline     for the dominant kernel of the step (the row-stream kernel
+               instantiation with the largest time per step), each projection
+               family's calls timed as a graph of their own, with every
+               family's figure and the gate/up call timed alone;
   cpu_baseline the fp64 oracle on the host, on a bounded sample of the step;
   secondary    every other workload's figures: the Gemma-3 dense comparator,
                the Gemma-3 G=1 rank-64 stacks at M = 1, 8, 64, the Gemma-4-31B
-               decode families at M = 1 and 16, the Gemma-4-31B prefill
+               decode families at M = 1 and 16 (bf16 W0, and NVFP4 W0 at M = 1),
+               the Gemma-4-31B prefill
                families (M = 4096), each a median over >= 1 s with p10 / p90
                and its fraction of the measured peak.
 With --gpus N > 1 each rank runs an independent replica (the path has no
@@ -335,6 +338,70 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
             "peak_source": peaks["source"]}
 
 
+def rows_instance(M, K, stacks):
+    """The row-stream kernel instantiation a call launches: (token tiles,
+    blocks per CTA, rank tiles), from the library's plan (None if the call
+    takes another kernel)."""
+    import linear_wl_forward_b200 as wl
+
+    try:
+        plan = wl.describe_rows_plan(M, K, stacks)
+    except wl.WLError:
+        return None
+    nb = plan["nb_max"]
+    rmax = max(r for _, r in stacks)
+    return ((M + 7) // 8, 1 if nb <= 1 else (2 if nb <= 2 else 4),
+            1 if rmax <= 16 else (2 if rmax <= 32 else 4))
+
+
+def sweep_roofline(wl, peaks, calls, dev_calls, outs, seconds):
+    """Roofline of the sweep's dominant kernel.  Each projection family's calls
+    of the step (26 layers, the bands' weights rotating) are timed as a graph
+    of their own; the kernel instantiation with the largest total time per
+    step is the dominant one, and its achieved bandwidth is its calls'
+    algorithmic bytes over their measured time."""
+    fams = {}
+    for i, c in enumerate(calls):
+        key = "+".join(p.family for p in c.projs)
+        fams.setdefault(key, []).append(i)
+    per = {}
+    for key, idx in fams.items():
+        c0 = calls[idx[0]]
+        M, K = c0.x.shape
+        stacks = [(p.N, p.r) for p in c0.projs]
+        g = capture(make_step([dev_calls[i] for i in idx], [outs[i] for i in idx], wl), 3)
+        st = per_call(time_windows(g, seconds), len(idx))
+        del g
+        b = sum(footprint.call_weight_bytes(p.N, p.K, p.r) for p in c0.projs) + \
+            footprint.call_io_bytes(M, sum(n for n, _ in stacks), K)
+        per[key] = {"instance": rows_instance(M, K, stacks), "bytes": b, "us": st["median_ms"] * 1e3,
+                    "us_p10": st["p10_ms"] * 1e3, "us_p90": st["p90_ms"] * 1e3, "calls_per_step": len(idx)}
+    groups = {}
+    for key, v in per.items():
+        groups.setdefault(v["instance"], []).append(key)
+    dom = max(groups, key=lambda k: sum(per[f]["us"] * per[f]["calls_per_step"] for f in groups[k]))
+    fb = sum(per[f]["bytes"] for f in groups[dom])
+    ft = sum(per[f]["us"] for f in groups[dom])
+    achieved = fb / (ft * 1e-6) / 1e9
+    kernel = f"rows_kernel<{dom[0]}, {dom[1]}, {dom[2]}>" if dom else "decode_kernel"
+    traffic = traffic_from_profile("rows_kernel", "gemma3_gate_up") if dom == (1, 4, 1) else None
+    return {"kernel": kernel + " (one launch per call: W0 x, V^T x, U T and the epilogue fused)",
+            "calls": "+".join(groups[dom]), "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "algorithmic_bytes": fb, "us_per_launch": round(ft / len(groups[dom]), 3),
+            "peak_source": peaks["source"],
+            "by_call": {k: {"kernel": f"rows_kernel<{v['instance'][0]}, {v['instance'][1]}, {v['instance'][2]}>"
+                            if v["instance"] else "decode_kernel",
+                            "algorithmic_bytes": v["bytes"], "us_per_launch": round(v["us"], 3),
+                            "us_p10": round(v["us_p10"], 3), "us_p90": round(v["us_p90"], 3),
+                            "GB/s": round(v["bytes"] / (v["us"] * 1e-6) / 1e9, 1),
+                            "frac": round(v["bytes"] / (v["us"] * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+                        for k, v in per.items()},
+            "how": "each family's 26 calls of the step as a graph of their own (CUDA events, windows "
+                   "over >= 1 s); achieved = the dominant instantiation's algorithmic bytes per "
+                   "launch (2NK + 2r(N+K) + 4N per projection, + x and y) over its launches' time"}
+
+
 def traffic_from_profile(kernel, call):
     """DRAM bytes per launch of `kernel` on `call` from the committed ncu
     summary, only while the kernel source is unchanged since the counters
@@ -429,6 +496,7 @@ def secondary_figures(wl, peaks, headline_ms, seconds):
             out[f"gemma4_decode_{name}_M{M}"] = rotating_figure(
                 wl, peaks, stacks, M, K, 3, seconds, ("g4d", name, M))
     out.update(gemma4_layer_figures(wl, peaks, seconds))
+    out.update(nvfp4_figures(wl, peaks, seconds))
     # Gemma-4-31B prefill, M = 4096: every family and the stacks
     g5 = {"q_sliding": ([(8192, 256)], 5376), "kv_sliding": ([(4096, 256)], 5376),
           "q_full": ([(16384, 256)], 5376), "k_full": ([(2048, 256)], 5376),
@@ -439,6 +507,47 @@ def secondary_figures(wl, peaks, headline_ms, seconds):
     for name, (stacks, K) in g5.items():
         out[f"gemma4_prefill_{name}_M4096"] = rotating_figure(
             wl, peaks, stacks, 4096, K, 1, seconds, ("g4p", name), kind="TFLOP/s")
+    return out
+
+
+def nvfp4_figures(wl, peaks, seconds):
+    """The NVFP4 decode path on the Gemma-4-31B decode families at M = 1
+    (rank 256, three distinct bundles per family, rotating): GB/s of the bytes
+    the call reads (codes, block scales, s, U, V), and the weight bytes per
+    token against the bf16 path's."""
+    from linear_wl_forward_b200 import footprint as fpt
+
+    fams = {"qkv_sliding": ([8192, 4096, 4096], 5376), "o_sliding": ([5376], 8192),
+            "qk_full": ([16384, 2048], 5376), "o_full": ([5376], 16384),
+            "gate_up": ([21504, 21504], 5376), "down": ([5376], 21504)}
+    out = {}
+    r = 256
+    for name, (Ns, K) in fams.items():
+        x = wl_inputs.device_x(1, K, "fp4", name)
+        dev = []
+        for c in range(3):
+            dev.append([wl_inputs.device_nvfp4_bundle(N, K, r, "fp4", name, c, i) for i, N in enumerate(Ns)])
+        outs = [[torch.empty(1, N, dtype=torch.bfloat16, device="cuda") for N in Ns] for _ in dev]
+
+        def step():
+            for projs, ys in zip(dev, outs):
+                wl.stacked_forward_nvfp4(x, projs, ys=ys)
+        g = capture(step, 3)
+        st = time_windows(g, seconds)
+        assert wl.last_device_status() == 0
+        per = per_call(st, len(dev))
+        ms = per["median_ms"]
+        read = sum(N * K // 2 + N * K // 16 + 4 * N + 2 * r * (N + K) for N in Ns)
+        bf16 = sum(fpt.call_weight_bytes(N, K, r) for N in Ns)
+        gbs = read / (ms * 1e-3) / 1e9
+        out[f"gemma4_decode_nvfp4_{name}_M1"] = {
+            "GB/s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+            "us_per_call": round(ms * 1e3, 2), "us_p10": round(per["p10_ms"] * 1e3, 2),
+            "us_p90": round(per["p90_ms"] * 1e3, 2), "bytes_read_per_call": read,
+            "bf16_path_weight_bytes_per_call": bf16, "bytes_ratio_vs_bf16": round(read / bf16, 4),
+            "launches_per_call": 2}
+        del g, dev, outs
+        torch.cuda.empty_cache()
     return out
 
 
@@ -743,7 +852,11 @@ def main():
     }
     if rank == 0 and world == 1:
         with ClockSampler(local) as clk2:
-            line["roofline"] = decode_roofline(wl, peaks, seconds=args.seconds)
+            if args.workload == "gemma3_decode":
+                line["roofline"] = sweep_roofline(wl, peaks, calls, dev_calls, outs, args.seconds)
+                line["roofline"]["gate_up_alone"] = decode_roofline(wl, peaks, seconds=args.seconds)
+            else:
+                line["roofline"] = decode_roofline(wl, peaks, seconds=args.seconds)
             if not args.no_secondary:
                 line["secondary"] = secondary_figures(wl, peaks, ms_step, args.seconds)
         line["secondary_clocks"] = clk2.summary()

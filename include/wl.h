@@ -211,6 +211,43 @@ wl_status wl_linear_forward_noalloc(const wl_bf16 *x, const wl_bf16 *W0, const f
  * array's address. */
 wl_status wl_noalloc_last_status(void *stream);
 
+/* One projection of an NVFP4 call: W0 stored as 4-bit codes with block
+ * scales, the encoding wl_quantize_nvfp4 produces ("Compression", "NVFP4:
+ * 3.18x smaller weights": packed 4-bit weights, one float8_e4m3fn scale per 16
+ * elements, 0.5625 bytes per element).  Device pointers. */
+typedef struct {
+    const uint8_t *codes;  /* N x K/2 bytes, row-major: FP4 E2M1, element 2i in the
+                              low nibble of byte i; 16-byte aligned             */
+    const uint8_t *scales; /* N x K/16 bytes, row-major: FP8 E4M3 scale of each
+                              16-element block along K; 2-byte aligned          */
+    float tensor_scale;    /* > 0: dequantised element = e2m1 * e4m3 * this     */
+    const float *s;        /* N                                              */
+    const wl_bf16 *U;      /* N x r row-major, 16-byte aligned (NULL iff r == 0) */
+    const wl_bf16 *V;      /* K x r row-major (NULL iff r == 0)                */
+    wl_bf16 *y;            /* M x N row-major (output)                         */
+    int N;                 /* output rows, >= 0                                */
+    int r;                 /* rank, 0 <= r <= WL_MAX_RANK, r % 8 == 0          */
+} wl_proj_nvfp4;
+
+#define WL_NVFP4_MAX_M 8
+
+/* The stacked forward with NVFP4 shared blocks: for each projection
+ *   y_p = s_p (.) (W0_p x) + U_p (V_p^T x),  W0_p the dequantised weight,
+ * computed as decode (1 <= M <= WL_NVFP4_MAX_M): the tensor scale multiplies
+ * s, the codes and block scales are expanded to f16 (an E2M1 value times an
+ * E4M3 scale is exact in f16) and multiplied with x rounded to f16 on the
+ * tensor cores, fp32 accumulation; U V^T x as in the bf16 path; y rounded once
+ * to bf16.  x is read as bf16 and rounded to f16 (round to nearest even),
+ * which is exact for |x| in [2^-14, 65504] -- the activations' range here.
+ * Two kernel launches (V^T x with x in f16, then the weight stream); scratch
+ * from the same pool as the other forward calls.  Errors: those of
+ * wl_stacked_forward; WL_ERR_ALIGNMENT unless K % 128 == 0, codes are 16-byte
+ * and scales 2-byte aligned, and every rank is a multiple of 8 with U 16-byte
+ * aligned; WL_ERR_INVALID_ARG for a tensor scale that is not > 0 and finite;
+ * WL_ERR_UNSUPPORTED for M > WL_NVFP4_MAX_M. */
+wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P,
+                                   void *stream);
+
 /* Host-side decomposition of L dense layer weights into theta bundles
  * ("Quality", "Why sharing fails": band-mean W0, per-row scale s, low-rank
  * residual; "Add a new model architecture", "Decompose HF weights" step 4).

@@ -12,7 +12,7 @@ import os
 
 __all__ = [
     "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
-    "prefetch_ranges", "MAX_PREFETCH",
+    "prefetch_ranges", "MAX_PREFETCH", "stacked_forward_nvfp4", "NVFP4_MAX_M",
     "materialize_weight", "describe_decode_plan", "DecodePlan", "describe_rows_plan", "RowsPlan",
     "quantize_nvfp4",
     "decompose",
@@ -30,6 +30,7 @@ DECODE_MAX_M = 16
 MAX_RANK = 1024
 MAX_PROJ = 8
 MAX_PREFETCH = 32
+NVFP4_MAX_M = 8
 
 
 class WLError(RuntimeError):
@@ -47,6 +48,12 @@ class _Proj(ctypes.Structure):
 
 class _Range(ctypes.Structure):
     _fields_ = [("ptr", ctypes.c_void_p), ("bytes", ctypes.c_size_t)]
+
+
+class _ProjNvfp4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_float),
+                ("s", ctypes.c_void_p), ("U", ctypes.c_void_p), ("V", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("N", ctypes.c_int), ("r", ctypes.c_int)]
 
 
 class RowsPlan(ctypes.Structure):
@@ -86,6 +93,7 @@ def lib():
         L.wl_materialize_weight.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, vp]
         L.wl_describe_decode_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci,
                                               ctypes.POINTER(DecodePlan)]
+        L.wl_stacked_forward_nvfp4.argtypes = [vp, ci, ci, ctypes.POINTER(_ProjNvfp4), ci, vp]
         L.wl_describe_rows_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci, ctypes.POINTER(RowsPlan)]
         L.wl_quantize_nvfp4.argtypes = [vp, ci, ci, ctypes.c_float, vp, vp, ctypes.POINTER(ctypes.c_float)]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
@@ -98,6 +106,7 @@ def lib():
         L.wl_noalloc_last_status.argtypes = [vp]
         L.wl_version.restype = ci
         for name in ("wl_linear_forward", "wl_stacked_forward", "wl_forward_ex", "wl_stacked_forward_prefetch",
+                     "wl_stacked_forward_nvfp4",
                      "wl_decompose", "wl_decompose_als",
                      "wl_materialize_weight", "wl_describe_decode_plan", "wl_describe_rows_plan",
                      "wl_quantize_nvfp4",
@@ -155,6 +164,31 @@ def linear_forward(x, W0, s, U, V, y=None, stream=None, path="auto"):
     bf16); asynchronous on `stream` (default: torch's current stream)."""
     return stacked_forward(x, [(W0, s, U, V)], ys=None if y is None else [y], stream=stream,
                            path=path)[0]
+
+
+def stacked_forward_nvfp4(x, projs, ys=None, stream=None):
+    """The stacked forward with NVFP4 shared blocks (include/wl.h,
+    wl_stacked_forward_nvfp4).  projs: (codes N x K/2 uint8, scales N x K/16
+    uint8, tensor_scale float, s, U, V) per projection, CUDA tensors (U = V =
+    None for r = 0).  Returns the list of y_p (M x N_p bf16)."""
+    import torch
+
+    M, K = x.shape
+    if ys is None:
+        ys = [torch.empty(M, c.shape[0], dtype=torch.bfloat16, device=x.device) for (c, *_rest) in projs]
+    arr = (_ProjNvfp4 * len(projs))()
+    for i, ((codes, scales, ts, s, U, V), y) in enumerate(zip(projs, ys)):
+        N = codes.shape[0]
+        r = 0 if U is None else U.shape[1]
+        arr[i] = _ProjNvfp4(_dev_ptr(codes, torch.uint8, "codes", (N, K // 2)),
+                            _dev_ptr(scales, torch.uint8, "scales", (N, K // 16)), float(ts),
+                            _dev_ptr(s, torch.float32, "s", (N,)),
+                            _dev_ptr(U, torch.bfloat16, "U", (N, r)) if r else None,
+                            _dev_ptr(V, torch.bfloat16, "V", (K, r)) if r else None,
+                            _dev_ptr(y, torch.bfloat16, "y", (M, N)), N, r)
+    _check(lib().wl_stacked_forward_nvfp4(_dev_ptr(x, torch.bfloat16, "x", (M, K)), M, K, arr, len(projs),
+                                          _stream_handle(stream)), "wl_stacked_forward_nvfp4")
+    return ys
 
 
 def prefetch_ranges(items):

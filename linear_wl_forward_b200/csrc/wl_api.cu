@@ -89,7 +89,11 @@ enum Slot {
     kSlotPart,
     kSlotTileCnt,  // zeroed when allocated; the kernels leave it zero
     kSlotUPad0,
-    kNumSlots = kSlotUPad0 + kMaxSeg
+    kSlotXh = kSlotUPad0 + kMaxSeg,  // NVFP4: x in f16
+    kSlotFp4Part,                    // NVFP4: partial sums of V^T x
+    kSlotFp4T,                       // NVFP4: V^T x
+    kSlotFp4Cnt,                     // NVFP4: prep CTAs done per projection (zeroed; self-resetting)
+    kNumSlots
 };
 
 struct DevicePool {
@@ -658,6 +662,90 @@ wl_status wl_describe_decode_plan(int M, int K, const wl_proj *projs, int P, int
     return WL_OK;
 }
 
+wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P,
+                                   void *stream_ptr) {
+    using namespace wl;
+    if (!projs) return WL_ERR_INVALID_ARG;
+    if (P < 1 || P > WL_MAX_PROJ) return P < 1 ? WL_ERR_INVALID_ARG : WL_ERR_UNSUPPORTED;
+    if (M < 0 || K < 0) return WL_ERR_INVALID_ARG;
+    bool any = false;
+    for (int i = 0; i < P; ++i) {
+        const wl_proj_nvfp4 &q = projs[i];
+        if (q.N < 0 || q.r < 0) return WL_ERR_INVALID_ARG;
+        if (q.r > WL_MAX_RANK) return WL_ERR_UNSUPPORTED;
+        if (q.N == 0) continue;
+        any = true;
+        if (M > 0 && (!q.y || !q.s || (K > 0 && (!q.codes || !q.scales)))) return WL_ERR_INVALID_ARG;
+        if (M > 0 && K > 0 && q.r > 0 && (!q.U || !q.V)) return WL_ERR_INVALID_ARG;
+        if (!(q.tensor_scale > 0.f) || !(q.tensor_scale < 3.0e38f)) return WL_ERR_INVALID_ARG;
+    }
+    if (M > 0 && K > 0 && !x) return WL_ERR_INVALID_ARG;
+    if (K % kFp4KGroup != 0) return WL_ERR_ALIGNMENT;
+    if (M > 0 && K > 0) {
+        if (!aligned16(x)) return WL_ERR_ALIGNMENT;
+        for (int i = 0; i < P; ++i) {
+            const wl_proj_nvfp4 &q = projs[i];
+            if (q.N == 0) continue;
+            if (!aligned16(q.codes) || (reinterpret_cast<uintptr_t>(q.scales) & 1u)) return WL_ERR_ALIGNMENT;
+            if (q.r > 0 && (q.r % 8 != 0 || !aligned16(q.U))) return WL_ERR_ALIGNMENT;
+        }
+    }
+    if (M > WL_NVFP4_MAX_M) return WL_ERR_UNSUPPORTED;
+    if (M == 0 || !any) return WL_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if (K == 0) {
+        for (int i = 0; i < P; ++i)
+            if (projs[i].N > 0 &&
+                cudaMemsetAsync(projs[i].y, 0, (size_t)M * projs[i].N * 2, stream) != cudaSuccess)
+                return WL_ERR_CUDA;
+        return WL_OK;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevicePool *pool = nullptr;
+    wl_status st = pool_for_current_device(&pool);
+    if (st != WL_OK) return st;
+    static Fp4Params fp;  // guarded by g_mu
+    std::memset(&fp, 0, sizeof fp);
+    int blocks = 0, t_off = 0, nr = 0;
+    for (int i = 0; i < P; ++i) {
+        const wl_proj_nvfp4 &q = projs[i];
+        if (q.N == 0) continue;
+        Fp4Seg &sg = fp.seg[fp.nseg++];
+        sg.codes = q.codes;
+        sg.scales = q.scales;
+        sg.ts = q.tensor_scale;
+        sg.s = q.s;
+        sg.U = reinterpret_cast<const __nv_bfloat16 *>(q.U);
+        sg.V = reinterpret_cast<const __nv_bfloat16 *>(q.V);
+        sg.y = reinterpret_cast<__nv_bfloat16 *>(q.y);
+        sg.N = q.N;
+        sg.r = q.r;
+        sg.blk_begin = blocks;
+        sg.t_off = t_off;
+        blocks += (q.N + 15) / 16;
+        t_off += q.r;
+        nr += q.r > 0;
+    }
+    fp.M = M;
+    fp.K = K;
+    fp.total_blocks = blocks;
+    fp.t_ld = t_off;
+    fp.slices = fp4_prep_slices(K);
+    fp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    void *xh = nullptr, *tp = nullptr, *tt = nullptr, *cnt = nullptr;
+    if ((st = scratch(*pool, kSlotXh, (size_t)M * K * 2, &xh)) != WL_OK) return st;
+    if ((st = scratch(*pool, kSlotFp4Part, fp4_tpart_floats(fp) * sizeof(float), &tp)) != WL_OK) return st;
+    if ((st = scratch(*pool, kSlotFp4T, (size_t)M * (t_off > 0 ? t_off : 1) * sizeof(float), &tt)) != WL_OK)
+        return st;
+    if ((st = scratch(*pool, kSlotFp4Cnt, (size_t)kMaxSeg * sizeof(unsigned), &cnt, true)) != WL_OK) return st;
+    fp.xh = static_cast<__half *>(xh);
+    fp.Tpart = static_cast<float *>(tp);
+    fp.T = static_cast<float *>(tt);
+    fp.cnt = static_cast<unsigned int *>(cnt);
+    (void)nr;
+    return from_cuda(launch_fp4(fp, stream));
+}
+
 wl_status wl_describe_rows_plan(int M, int K, const wl_proj *projs, int P, int num_sms, wl_rows_plan *out) {
     if (!out || num_sms < 1) return WL_ERR_INVALID_ARG;
     std::memset(out, 0, sizeof *out);
@@ -688,9 +776,9 @@ wl_status wl_last_device_status(void *stream) {
     // A kernel that gave up may have left its arrival counters set: clear the
     // whole word block (status and counters) after an error.
     if (word != 0 && cudaMemset(pool->words, 0, 64 * sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
-    if (word != 0 && pool->buf[wl::kSlotTileCnt] &&
-        cudaMemset(pool->buf[wl::kSlotTileCnt], 0, pool->cap[wl::kSlotTileCnt]) != cudaSuccess)
-        return WL_ERR_CUDA;
+    for (int slot : {(int)wl::kSlotTileCnt, (int)wl::kSlotFp4Cnt})
+        if (word != 0 && pool->buf[slot] && cudaMemset(pool->buf[slot], 0, pool->cap[slot]) != cudaSuccess)
+            return WL_ERR_CUDA;
     return static_cast<wl_status>(word);
 }
 

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -180,6 +181,44 @@ struct RowsParams {
 wl_status plan_rows(RowsParams &p, int M, int K, const wl_proj *projs, int P, int num_sms,
                     bool encode_maps = true);
 cudaError_t launch_rows(const RowsParams &p, cudaStream_t stream);
+
+// -------------------------------------------------------- NVFP4 decode ----
+// Decode with W0 stored as NVFP4 (E2M1 codes, E4M3 scales per 16 elements,
+// fp32 tensor scale): a prep launch forms T = V^T x and x in f16, a stream
+// launch runs one CTA per 16-row block of W0.
+constexpr int kFp4KGroup = 128;  // K columns per warp step; K must be a multiple
+constexpr int kFp4MaxM = 8;      // tokens
+
+struct Fp4Seg {
+    const uint8_t *codes;   // N x K/2
+    const uint8_t *scales;  // N x K/16
+    float ts;               // tensor scale
+    const float *s;
+    const __nv_bfloat16 *U;
+    const __nv_bfloat16 *V;
+    __nv_bfloat16 *y;
+    int N, r;
+    int blk_begin;  // first 16-row block of this projection
+    int t_off;      // column of this projection's slice in T
+};
+
+struct Fp4Params {
+    Fp4Seg seg[kMaxSeg];
+    int nseg;
+    int M, K;
+    int total_blocks;
+    int t_ld;     // sum of ranks
+    int slices;   // prep CTAs per projection with a delta (K slices)
+    const __nv_bfloat16 *x;
+    __half *xh;          // M x K, x in f16 (written by the prep launch)
+    float *Tpart;        // per projection [slices][M][r] partial sums
+    float *T;            // [M][t_ld]
+    unsigned int *cnt;   // per projection slot: prep CTAs done (zeroed at allocation, self-resetting)
+};
+
+int fp4_prep_slices(int K);
+size_t fp4_tpart_floats(const Fp4Params &p);
+cudaError_t launch_fp4(const Fp4Params &p, cudaStream_t stream);
 
 // ----------------------------------------------------------------- GEMM ----
 // tcgen05 GEMM: Y[m][n] = s[n] * sum_k A[m][k] B[n][k] + sum_j T[m][j] U[n][j].

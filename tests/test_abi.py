@@ -120,3 +120,23 @@ def test_wait_limit_validation(L):
     assert L.wl_set_wait_limit(20_000_000_000) == 1
     assert L.wl_set_wait_limit(1000) == 0
     assert L.wl_set_wait_limit(0) == 0  # back to the default
+
+
+def test_nvfp4_validation(L):
+    """wl_stacked_forward_nvfp4 rejects bad calls on the host."""
+    def call(M=1, K=128, N=16, r=8, ts=0.5, codes=FAKE, scales=FAKE, U=FAKE):
+        arr = (wl._ProjNvfp4 * 1)(wl._ProjNvfp4(codes, scales, ts, FAKE, U, FAKE, FAKE, N, r))
+        return L.wl_stacked_forward_nvfp4(FAKE, M, K, arr, 1, None)
+
+    assert call(K=64) == 2                 # K % 128
+    assert call(codes=FAKE + 8) == 2       # codes 16-byte aligned
+    assert call(scales=FAKE + 1) == 2      # scales 2-byte aligned
+    assert call(r=12) == 2                 # rank % 8
+    assert call(U=FAKE + 8) == 2           # U 16-byte aligned
+    assert call(ts=0.0) == 1
+    assert call(ts=-1.0) == 1
+    assert call(ts=float("inf")) == 1
+    assert call(M=wl.NVFP4_MAX_M + 1) == 3
+    assert call(r=wl.MAX_RANK + 8) == 3
+    assert call(M=0) == 0                  # empty calls touch nothing
+    assert L.wl_stacked_forward_nvfp4(FAKE, 1, 128, None, 1, None) == 1

@@ -293,3 +293,18 @@ def device_x(M: int, K: int, *key, device="cuda"):
     g = torch.Generator(device=device)
     g.manual_seed(subseed("device-x", *key))
     return torch.randn(M, K, generator=g, device=device).to(torch.bfloat16)
+
+
+def device_nvfp4_bundle(N: int, K: int, r: int, *key, device="cuda"):
+    """(codes N x K/2 uint8, scale bytes N x K/16 uint8, tensor scale, s, U, V)
+    of an NVFP4 projection drawn on `device` for timing runs: uniformly random
+    code bytes, scale bytes in 0x30 .. 0x4F (E4M3 0.5 .. 15), the tensor scale
+    of draw_w0_nvfp4; s, U, V as device_bundle."""
+    g = torch.Generator(device=device)
+    g.manual_seed(subseed("device-nvfp4", *key))
+    codes = torch.randint(0, 256, (N, K // 2), generator=g, device=device, dtype=torch.uint8)
+    scales = torch.randint(0x30, 0x50, (N, K // 16), generator=g, device=device, dtype=torch.uint8)
+    s = torch.rand(N, generator=g, device=device) * (S_HI - S_LO) + S_LO
+    U = (torch.randn(N, r, generator=g, device=device) * W_STD).to(torch.bfloat16) if r else None
+    V = (torch.randn(K, r, generator=g, device=device) * W_STD).to(torch.bfloat16) if r else None
+    return codes, scales, NVFP4_TENSOR_SCALE, s, U, V
