@@ -223,7 +223,7 @@ typedef struct {
     float tensor_scale;    /* > 0: dequantised element = e2m1 * e4m3 * this     */
     const float *s;        /* N                                              */
     const wl_bf16 *U;      /* N x r row-major, 16-byte aligned (NULL iff r == 0) */
-    const wl_bf16 *V;      /* K x r row-major (NULL iff r == 0)                */
+    const wl_bf16 *V;      /* K x r row-major, 16-byte aligned (NULL iff r == 0) */
     wl_bf16 *y;            /* M x N row-major (output)                         */
     int N;                 /* output rows, >= 0                                */
     int r;                 /* rank, 0 <= r <= WL_MAX_RANK, r % 8 == 0          */
@@ -239,14 +239,38 @@ typedef struct {
  * tensor cores, fp32 accumulation; U V^T x as in the bf16 path; y rounded once
  * to bf16.  x is read as bf16 and rounded to f16 (round to nearest even),
  * which is exact for |x| in [2^-14, 65504] -- the activations' range here.
- * Two kernel launches (V^T x with x in f16, then the weight stream); scratch
- * from the same pool as the other forward calls.  Errors: those of
+ * Two kernel launches (V^T x with x in f16, then the weight stream: a
+ * persistent TMA ring over all SMs when K % 256 == 0, every rank is at most
+ * 256 and every scales pointer is 16-byte aligned, else one CTA per 16 rows);
+ * scratch from the same pool as the other forward calls.  Results are
+ * reproducible for a given call shape and GPU.  Errors: those of
  * wl_stacked_forward; WL_ERR_ALIGNMENT unless K % 128 == 0, codes are 16-byte
- * and scales 2-byte aligned, and every rank is a multiple of 8 with U 16-byte
- * aligned; WL_ERR_INVALID_ARG for a tensor scale that is not > 0 and finite;
- * WL_ERR_UNSUPPORTED for M > WL_NVFP4_MAX_M. */
+ * and scales 2-byte aligned, and every rank is a multiple of 8 with U and V
+ * 16-byte aligned; WL_ERR_INVALID_ARG for a tensor scale that is not > 0 and
+ * finite; WL_ERR_UNSUPPORTED for M > WL_NVFP4_MAX_M.  Device-side waits are
+ * bounded as in the other calls (wl_last_device_status). */
 wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P,
                                    void *stream);
+
+/* What wl_stacked_forward_nvfp4 would launch for a call: the host-side plan,
+ * made without a GPU (no tensor maps, no launch).  The pointers in `projs` are
+ * only checked (null, alignment), never dereferenced; `num_sms` stands for the
+ * device's SM count.  Errors as wl_stacked_forward_nvfp4's argument checks;
+ * all-zero for a call with nothing to launch. */
+typedef struct {
+    int ring;          /* 1: persistent TMA ring stream, 0: one CTA per 16 rows */
+    int grid;          /* CTAs of the weight stream                            */
+    int stages;        /* ring slots per CTA (ring only)                       */
+    int slot_bytes;    /* bytes of one ring slot (ring only)                   */
+    int smem_bytes;    /* dynamic shared memory per CTA (ring only)            */
+    long long units;   /* (block, stage) units split over the CTAs (ring only) */
+    int prep_slices;   /* slices of K in the V^T x launch                      */
+    int prep_rows;     /* rows of V per slice                                  */
+    int prep_grid;     /* CTAs of the V^T x launch                             */
+} wl_nvfp4_plan;
+
+wl_status wl_describe_nvfp4_plan(int M, int K, const wl_proj_nvfp4 *projs, int P, int num_sms,
+                                 wl_nvfp4_plan *out);
 
 /* Host-side decomposition of L dense layer weights into theta bundles
  * ("Quality", "Why sharing fails": band-mean W0, per-row scale s, low-rank

@@ -14,6 +14,7 @@ __all__ = [
     "WLError", "lib", "linear_forward", "stacked_forward", "prepare_stacked", "PreparedForward",
     "prefetch_ranges", "MAX_PREFETCH", "stacked_forward_nvfp4", "NVFP4_MAX_M",
     "materialize_weight", "describe_decode_plan", "DecodePlan", "describe_rows_plan", "RowsPlan",
+    "describe_nvfp4_plan", "Nvfp4Plan",
     "quantize_nvfp4",
     "decompose",
     "relative_frobenius_error", "last_device_status", "wait_probe", "set_wait_limit", "PATHS",
@@ -62,6 +63,13 @@ class RowsPlan(ctypes.Structure):
                 ("nb_max", ctypes.c_int), ("k_slice", ctypes.c_int), ("smem_bytes", ctypes.c_longlong)]
 
 
+class Nvfp4Plan(ctypes.Structure):
+    """wl_nvfp4_plan of include/wl.h."""
+    _fields_ = [("ring", ctypes.c_int), ("grid", ctypes.c_int), ("stages", ctypes.c_int),
+                ("slot_bytes", ctypes.c_int), ("smem_bytes", ctypes.c_int), ("units", ctypes.c_longlong),
+                ("prep_slices", ctypes.c_int), ("prep_rows", ctypes.c_int), ("prep_grid", ctypes.c_int)]
+
+
 class DecodePlan(ctypes.Structure):
     """wl_decode_plan of include/wl.h."""
     _fields_ = [("auto_decode", ctypes.c_int), ("grid", ctypes.c_int), ("compact", ctypes.c_int),
@@ -95,6 +103,7 @@ def lib():
                                               ctypes.POINTER(DecodePlan)]
         L.wl_stacked_forward_nvfp4.argtypes = [vp, ci, ci, ctypes.POINTER(_ProjNvfp4), ci, vp]
         L.wl_describe_rows_plan.argtypes = [ci, ci, ctypes.POINTER(_Proj), ci, ci, ctypes.POINTER(RowsPlan)]
+        L.wl_describe_nvfp4_plan.argtypes = [ci, ci, ctypes.POINTER(_ProjNvfp4), ci, ci, ctypes.POINTER(Nvfp4Plan)]
         L.wl_quantize_nvfp4.argtypes = [vp, ci, ci, ctypes.c_float, vp, vp, ctypes.POINTER(ctypes.c_float)]
         L.wl_relative_frobenius_error.argtypes = [vp] * 5 + [ci] * 3
         L.wl_relative_frobenius_error.restype = ctypes.c_double
@@ -109,6 +118,7 @@ def lib():
                      "wl_stacked_forward_nvfp4",
                      "wl_decompose", "wl_decompose_als",
                      "wl_materialize_weight", "wl_describe_decode_plan", "wl_describe_rows_plan",
+                     "wl_describe_nvfp4_plan",
                      "wl_quantize_nvfp4",
                      "wl_last_device_status", "wl_wait_probe", "wl_set_wait_limit", "wl_noalloc_last_status"):
             getattr(L, name).restype = ci
@@ -352,6 +362,25 @@ def describe_rows_plan(M: int, K: int, projs, num_sms: int = 148) -> dict:
     _check(lib().wl_describe_rows_plan(M, K, arr, len(projs), num_sms, ctypes.byref(out)),
            "wl_describe_rows_plan")
     return {name: getattr(out, name) for name, _ in RowsPlan._fields_}
+
+
+def describe_nvfp4_plan(M: int, K: int, projs, num_sms: int = 148) -> dict:
+    """The NVFP4 forward's host-side plan for a call, made without a GPU.
+    ``projs``: (N, r) or (N, r, scales_offset_bytes) per projection; stand-in
+    addresses (never dereferenced) are 16-byte aligned, the scales moved by
+    the offset."""
+    arr = (_ProjNvfp4 * len(projs))()
+    for i, q in enumerate(projs):
+        N, r = q[0], q[1]
+        off = q[2] if len(q) > 2 else 0
+        base = (i + 1) << 32
+        arr[i] = _ProjNvfp4(base, base + (1 << 28) + off, 1.0, base + (2 << 28),
+                            (base + (3 << 28)) if r else None, (base + (4 << 28)) if r else None,
+                            base + (5 << 28), N, r)
+    out = Nvfp4Plan()
+    _check(lib().wl_describe_nvfp4_plan(M, K, arr, len(projs), num_sms, ctypes.byref(out)),
+           "wl_describe_nvfp4_plan")
+    return {name: getattr(out, name) for name, _ in Nvfp4Plan._fields_}
 
 
 def last_device_status(stream=None) -> int:

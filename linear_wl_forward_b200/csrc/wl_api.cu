@@ -55,17 +55,45 @@ wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t
     return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
 }
 
+wl_status encode_map_2d_u32(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld_bytes,
+                            uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return WL_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
+}
+
+wl_status encode_map_1d_f32(CUtensorMap *m, const void *ptr, uint64_t n, uint32_t box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return WL_ERR_CUDA;
+    const cuuint64_t dims[1] = {n};
+    const cuuint64_t strides[1] = {n * 4};  // not read for a rank-1 map
+    const cuuint32_t bx[1] = {box};
+    const cuuint32_t estr[1] = {1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<void *>(ptr), dims, strides, bx, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
+}
+
 wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                         uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
-                        uint32_t b2) {
+                        uint32_t b2, bool bytes_unswizzled) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return WL_ERR_CUDA;
     const cuuint64_t dims[3] = {d0, d1, d2};
     const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
     const cuuint32_t box[3] = {b0, b1, b2};
     const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
-                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUresult r = fn(m, bytes_unswizzled ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                          const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          bytes_unswizzled ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? WL_OK : WL_ERR_CUDA;
 }
@@ -89,10 +117,13 @@ enum Slot {
     kSlotPart,
     kSlotTileCnt,  // zeroed when allocated; the kernels leave it zero
     kSlotUPad0,
-    kSlotXh = kSlotUPad0 + kMaxSeg,  // NVFP4: x in f16
-    kSlotFp4Part,                    // NVFP4: partial sums of V^T x
+    kSlotXh = kSlotUPad0 + kMaxSeg,  // NVFP4: permuted x in f16
+    kSlotFp4Part,                    // NVFP4: slice partial sums of V^T x
     kSlotFp4T,                       // NVFP4: V^T x
-    kSlotFp4Cnt,                     // NVFP4: prep CTAs done per projection (zeroed; self-resetting)
+    kSlotFp4Cnt,                     // NVFP4: prep group / projection counters (zeroed; self-resetting)
+    kSlotFp4G,                       // NVFP4: group sums of V^T x
+    kSlotFp4Blk,                     // NVFP4 ring: partial sums of blocks split between CTAs
+    kSlotFp4BCnt,                    // NVFP4 ring: CTAs done per split block (zeroed; self-resetting)
     kNumSlots
 };
 
@@ -662,9 +693,13 @@ wl_status wl_describe_decode_plan(int M, int K, const wl_proj *projs, int P, int
     return WL_OK;
 }
 
-wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P,
-                                   void *stream_ptr) {
+namespace {
+
+// Argument checks of the NVFP4 forward; WL_OK with *trivial set when there is
+// nothing to launch (M == 0, no rows, or K == 0).
+wl_status nvfp4_validate(const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P, bool *trivial) {
     using namespace wl;
+    *trivial = false;
     if (!projs) return WL_ERR_INVALID_ARG;
     if (P < 1 || P > WL_MAX_PROJ) return P < 1 ? WL_ERR_INVALID_ARG : WL_ERR_UNSUPPORTED;
     if (M < 0 || K < 0) return WL_ERR_INVALID_ARG;
@@ -687,24 +722,17 @@ wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj
             const wl_proj_nvfp4 &q = projs[i];
             if (q.N == 0) continue;
             if (!aligned16(q.codes) || (reinterpret_cast<uintptr_t>(q.scales) & 1u)) return WL_ERR_ALIGNMENT;
-            if (q.r > 0 && (q.r % 8 != 0 || !aligned16(q.U))) return WL_ERR_ALIGNMENT;
+            if (q.r > 0 && (q.r % 8 != 0 || !aligned16(q.U) || !aligned16(q.V))) return WL_ERR_ALIGNMENT;
         }
     }
     if (M > WL_NVFP4_MAX_M) return WL_ERR_UNSUPPORTED;
-    if (M == 0 || !any) return WL_OK;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-    if (K == 0) {
-        for (int i = 0; i < P; ++i)
-            if (projs[i].N > 0 &&
-                cudaMemsetAsync(projs[i].y, 0, (size_t)M * projs[i].N * 2, stream) != cudaSuccess)
-                return WL_ERR_CUDA;
-        return WL_OK;
-    }
-    std::lock_guard<std::mutex> lock(g_mu);
-    DevicePool *pool = nullptr;
-    wl_status st = pool_for_current_device(&pool);
-    if (st != WL_OK) return st;
-    static Fp4Params fp;  // guarded by g_mu
+    *trivial = M == 0 || !any || K == 0;
+    return WL_OK;
+}
+
+// The projections with rows, in order, as kernel segments.
+void nvfp4_fill(wl::Fp4Params &fp, const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P) {
+    using namespace wl;
     std::memset(&fp, 0, sizeof fp);
     int blocks = 0, t_off = 0, nr = 0;
     for (int i = 0; i < P; ++i) {
@@ -730,20 +758,85 @@ wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj
     fp.K = K;
     fp.total_blocks = blocks;
     fp.t_ld = t_off;
-    fp.slices = fp4_prep_slices(K);
+    fp.nr = nr;
     fp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-    void *xh = nullptr, *tp = nullptr, *tt = nullptr, *cnt = nullptr;
-    if ((st = scratch(*pool, kSlotXh, (size_t)M * K * 2, &xh)) != WL_OK) return st;
-    if ((st = scratch(*pool, kSlotFp4Part, fp4_tpart_floats(fp) * sizeof(float), &tp)) != WL_OK) return st;
-    if ((st = scratch(*pool, kSlotFp4T, (size_t)M * (t_off > 0 ? t_off : 1) * sizeof(float), &tt)) != WL_OK)
+}
+
+}  // namespace
+
+wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj_nvfp4 *projs, int P,
+                                   void *stream_ptr) {
+    using namespace wl;
+    bool trivial = false;
+    wl_status st = nvfp4_validate(x, M, K, projs, P, &trivial);
+    if (st != WL_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    if (trivial) {
+        if (M > 0 && K == 0)
+            for (int i = 0; i < P; ++i)
+                if (projs[i].N > 0 &&
+                    cudaMemsetAsync(projs[i].y, 0, (size_t)M * projs[i].N * 2, stream) != cudaSuccess)
+                    return WL_ERR_CUDA;
+        return WL_OK;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevicePool *pool = nullptr;
+    if ((st = pool_for_current_device(&pool)) != WL_OK) return st;
+    static Fp4Params fp;  // guarded by g_mu
+    nvfp4_fill(fp, x, M, K, projs, P);
+    fp.status = pool->words;
+    fp.timeout_ns = wait_limit_ns();
+    if ((st = plan_fp4(fp, pool->num_sms)) != WL_OK) return st;
+    const size_t tl = (size_t)(fp.t_ld > 0 ? fp.t_ld : 1);
+    void *xq = nullptr, *tp = nullptr, *gp = nullptr, *tt = nullptr, *cnt = nullptr;
+    if ((st = scratch(*pool, kSlotXh, fp4_xq_halves(fp) * 2, &xq)) != WL_OK) return st;
+    if ((st = scratch(*pool, kSlotFp4Part, (size_t)fp.slices * M * tl * sizeof(float), &tp)) != WL_OK) return st;
+    if ((st = scratch(*pool, kSlotFp4G, (size_t)fp.ngrp * M * tl * sizeof(float), &gp)) != WL_OK) return st;
+    if ((st = scratch(*pool, kSlotFp4T, (size_t)M * tl * sizeof(float), &tt)) != WL_OK) return st;
+    if ((st = scratch(*pool, kSlotFp4Cnt, (size_t)(kMaxSeg * (fp.ngrp + 1)) * sizeof(unsigned), &cnt, true)) !=
+        WL_OK)
         return st;
-    if ((st = scratch(*pool, kSlotFp4Cnt, (size_t)kMaxSeg * sizeof(unsigned), &cnt, true)) != WL_OK) return st;
-    fp.xh = static_cast<__half *>(xh);
+    fp.xq = static_cast<__half *>(xq);
     fp.Tpart = static_cast<float *>(tp);
+    fp.Gpart = static_cast<float *>(gp);
     fp.T = static_cast<float *>(tt);
     fp.cnt = static_cast<unsigned int *>(cnt);
-    (void)nr;
+    if (fp.ring) {
+        void *pa = nullptr, *bc = nullptr;
+        if ((st = scratch(*pool, kSlotFp4Blk, (size_t)fp.grid * 2 * 16 * kFp4MaxM * sizeof(float2), &pa)) != WL_OK)
+            return st;
+        if ((st = scratch(*pool, kSlotFp4BCnt, (size_t)fp.total_blocks * sizeof(unsigned), &bc, true)) != WL_OK)
+            return st;
+        fp.parts = static_cast<float2 *>(pa);
+        fp.bcnt = static_cast<unsigned int *>(bc);
+    }
     return from_cuda(launch_fp4(fp, stream));
+}
+
+wl_status wl_describe_nvfp4_plan(int M, int K, const wl_proj_nvfp4 *projs, int P, int num_sms,
+                                 wl_nvfp4_plan *out) {
+    using namespace wl;
+    if (!out || num_sms < 1) return WL_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof *out);
+    alignas(16) static const unsigned char no_x[16] = {};
+    bool trivial = false;
+    wl_status st = nvfp4_validate(reinterpret_cast<const wl_bf16 *>(no_x), M, K, projs, P, &trivial);
+    if (st != WL_OK) return st;
+    if (trivial) return WL_OK;
+    static Fp4Params fp;  // guarded by g_mu
+    std::lock_guard<std::mutex> lock(g_mu);
+    nvfp4_fill(fp, reinterpret_cast<const wl_bf16 *>(no_x), M, K, projs, P);
+    if ((st = plan_fp4(fp, num_sms, false)) != WL_OK) return st;
+    out->ring = fp.ring;
+    out->grid = fp.ring ? fp.grid : fp.total_blocks;
+    out->stages = fp.ring ? fp.ns : 0;
+    out->slot_bytes = fp.ring ? fp.slot_bytes : 0;
+    out->smem_bytes = fp.ring ? fp.smem : 0;
+    out->units = fp.ring ? fp.utot : 0;
+    out->prep_slices = fp.slices;
+    out->prep_rows = fp.kr;
+    out->prep_grid = fp.slices * (fp.nr > 0 ? fp.nr : 1);
+    return WL_OK;
 }
 
 wl_status wl_describe_rows_plan(int M, int K, const wl_proj *projs, int P, int num_sms, wl_rows_plan *out) {
@@ -776,7 +869,7 @@ wl_status wl_last_device_status(void *stream) {
     // A kernel that gave up may have left its arrival counters set: clear the
     // whole word block (status and counters) after an error.
     if (word != 0 && cudaMemset(pool->words, 0, 64 * sizeof(int)) != cudaSuccess) return WL_ERR_CUDA;
-    for (int slot : {(int)wl::kSlotTileCnt, (int)wl::kSlotFp4Cnt})
+    for (int slot : {(int)wl::kSlotTileCnt, (int)wl::kSlotFp4Cnt, (int)wl::kSlotFp4BCnt})
         if (word != 0 && pool->buf[slot] && cudaMemset(pool->buf[slot], 0, pool->cap[slot]) != cudaSuccess)
             return WL_ERR_CUDA;
     return static_cast<wl_status>(word);

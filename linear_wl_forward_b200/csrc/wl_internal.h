@@ -124,9 +124,15 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, cudaStr
 // out-of-range reads give 0.
 wl_status encode_map_2d(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld,
                         uint32_t box_cols, uint32_t box_rows, bool swizzle128 = true);
+// Raw bytes viewed as 32-bit words: rows of `cols` words, `ld_bytes` apart
+// (a multiple of 16), no swizzle.
+wl_status encode_map_2d_u32(CUtensorMap *m, const void *ptr, uint64_t cols, uint64_t rows, uint64_t ld_bytes,
+                            uint32_t box_cols, uint32_t box_rows);
+// n fp32 values, boxes of `box`.
+wl_status encode_map_1d_f32(CUtensorMap *m, const void *ptr, uint64_t n, uint32_t box);
 wl_status encode_map_3d(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                         uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
-                        uint32_t b2);
+                        uint32_t b2, bool bytes_unswizzled = false);
 
 // ----------------------------------------------------------- row stream ----
 // Row-stream decode kernel for short calls (latency-bound: a few MB of
@@ -184,10 +190,18 @@ cudaError_t launch_rows(const RowsParams &p, cudaStream_t stream);
 
 // -------------------------------------------------------- NVFP4 decode ----
 // Decode with W0 stored as NVFP4 (E2M1 codes, E4M3 scales per 16 elements,
-// fp32 tensor scale): a prep launch forms T = V^T x and x in f16, a stream
-// launch runs one CTA per 16-row block of W0.
+// fp32 tensor scale).  A prep launch forms T = V^T x and a permuted f16 copy
+// of x; then one of two weight-stream launches:
+//  * ring (K % 256 == 0, every rank <= 256): persistent, one CTA per SM; a
+//    producer warp streams (block, stage) units through a shared-memory ring
+//    by TMA, the units split evenly over the CTAs;
+//  * blocks (otherwise): one CTA per 16-row block, loads straight into
+//    registers.
 constexpr int kFp4KGroup = 128;  // K columns per warp step; K must be a multiple
 constexpr int kFp4MaxM = 8;      // tokens
+constexpr int kFp4StageKG = 16;  // k-groups per ring stage (2048 columns)
+constexpr int kFp4RingMaxRank = 256;
+constexpr int kFp4RingMaxStages = 16;
 
 struct Fp4Seg {
     const uint8_t *codes;   // N x K/2
@@ -200,24 +214,47 @@ struct Fp4Seg {
     int N, r;
     int blk_begin;  // first 16-row block of this projection
     int t_off;      // column of this projection's slice in T
+    long long ub;   // ring: first unit of this projection
+    int upb;        // ring: units per block (stages, plus one for U when r > 0)
 };
 
 struct Fp4Params {
     Fp4Seg seg[kMaxSeg];
+    CUtensorMap tm_c[kMaxSeg];  // ring: codes as 32-bit words, box 16 rows x 512 bytes
+    CUtensorMap tm_s[kMaxSeg];  // ring: scales as 32-bit words, box 16 rows x 64 bytes
+    CUtensorMap tm_u[kMaxSeg];  // ring: U as 32-bit words, box 16 rows x 2r bytes
+    CUtensorMap tm_sv[kMaxSeg]; // ring: s, boxes of 16 values
     int nseg;
     int M, K;
+    int Mp;       // token rows of the permuted x (M, rounded up to even above 1)
     int total_blocks;
     int t_ld;     // sum of ranks
-    int slices;   // prep CTAs per projection with a delta (K slices)
+    int nr;       // projections with a delta
+    // prep: T over slices of K, summed in groups of kFp4GroupSlices then over groups
+    int slices, kr, ngrp;
     const __nv_bfloat16 *x;
-    __half *xh;          // M x K, x in f16 (written by the prep launch)
-    float *Tpart;        // per projection [slices][M][r] partial sums
-    float *T;            // [M][t_ld]
-    unsigned int *cnt;   // per projection slot: prep CTAs done (zeroed at allocation, self-resetting)
+    __half *xq;           // permuted f16 x (written by the prep launch)
+    float *Tpart;         // [slices][M][t_ld]
+    float *Gpart;         // [ngrp][M][t_ld]
+    float *T;             // [M][t_ld]
+    unsigned int *cnt;    // [nr][ngrp] group counters, then [nr] projection counters (zeroed, self-resetting)
+    // ring
+    int ring;             // 1: ring stream, 0: block stream
+    int grid, ns, slot_bytes, smem, nst;
+    long long utot;
+    float2 *parts;        // [grid][2][16 * kFp4MaxM] partial (z, d) of blocks split between CTAs
+    unsigned int *bcnt;   // [total_blocks] CTAs done with a split block (zeroed, self-resetting)
+    int *status;
+    unsigned long long timeout_ns;
 };
 
-int fp4_prep_slices(int K);
-size_t fp4_tpart_floats(const Fp4Params &p);
+constexpr int kFp4GroupSlices = 16;
+constexpr int kFp4PrepMaxRows = 256;
+
+// Fills slices/kr/ngrp/Mp and, for the ring stream (encode_maps), the tensor
+// maps and ring geometry; p.seg/nseg/M/K/t_ld/nr must be set.
+wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps = true);
+size_t fp4_xq_halves(const Fp4Params &p);
 cudaError_t launch_fp4(const Fp4Params &p, cudaStream_t stream);
 
 // ----------------------------------------------------------------- GEMM ----

@@ -124,8 +124,8 @@ def test_wait_limit_validation(L):
 
 def test_nvfp4_validation(L):
     """wl_stacked_forward_nvfp4 rejects bad calls on the host."""
-    def call(M=1, K=128, N=16, r=8, ts=0.5, codes=FAKE, scales=FAKE, U=FAKE):
-        arr = (wl._ProjNvfp4 * 1)(wl._ProjNvfp4(codes, scales, ts, FAKE, U, FAKE, FAKE, N, r))
+    def call(M=1, K=128, N=16, r=8, ts=0.5, codes=FAKE, scales=FAKE, U=FAKE, V=FAKE):
+        arr = (wl._ProjNvfp4 * 1)(wl._ProjNvfp4(codes, scales, ts, FAKE, U, V, FAKE, N, r))
         return L.wl_stacked_forward_nvfp4(FAKE, M, K, arr, 1, None)
 
     assert call(K=64) == 2                 # K % 128
@@ -133,6 +133,7 @@ def test_nvfp4_validation(L):
     assert call(scales=FAKE + 1) == 2      # scales 2-byte aligned
     assert call(r=12) == 2                 # rank % 8
     assert call(U=FAKE + 8) == 2           # U 16-byte aligned
+    assert call(V=FAKE + 8) == 2           # V 16-byte aligned
     assert call(ts=0.0) == 1
     assert call(ts=-1.0) == 1
     assert call(ts=float("inf")) == 1
@@ -140,3 +141,31 @@ def test_nvfp4_validation(L):
     assert call(r=wl.MAX_RANK + 8) == 3
     assert call(M=0) == 0                  # empty calls touch nothing
     assert L.wl_stacked_forward_nvfp4(FAKE, 1, 128, None, 1, None) == 1
+
+
+def test_nvfp4_plan_picks_the_stream():
+    """wl_describe_nvfp4_plan: the ring stream for K % 256 == 0, K >= 16384,
+    ranks <= 256, 16-byte-aligned scales and at most 4 row blocks per SM; one
+    CTA per 16-row block otherwise.  The ring's shared memory fits a CTA and its
+    units cover the call."""
+    ring = wl.describe_nvfp4_plan(1, 21504, [(5376, 256)])      # Gemma-4 down
+    assert ring["ring"] == 1 and ring["grid"] == 148
+    assert ring["units"] == 336 * (11 + 1)           # 336 blocks x (11 stages of 2048 columns + U) each
+    assert ring["smem_bytes"] <= 227 * 1024 and ring["stages"] >= 4
+    assert ring["prep_grid"] == ring["prep_slices"]
+    assert ring["prep_slices"] * ring["prep_rows"] >= 21504
+    gate_up = wl.describe_nvfp4_plan(1, 5376, [(21504, 256), (21504, 256)])
+    assert gate_up["ring"] == 0 and gate_up["grid"] == 2 * 1344   # 2688 blocks > 4 per SM
+    assert gate_up["prep_grid"] == 2 * gate_up["prep_slices"]
+    assert wl.describe_nvfp4_plan(1, 8192, [(5376, 256)])["ring"] == 0       # Gemma-4 o: K < 16384
+    for M in range(1, wl.NVFP4_MAX_M + 1):
+        p = wl.describe_nvfp4_plan(M, 16384, [(700, 256)])
+        assert p["ring"] == 1 and p["smem_bytes"] <= 227 * 1024 and p["stages"] >= 4
+    assert wl.describe_nvfp4_plan(1, 1152, [(300, 16)])["ring"] == 0          # K % 256 != 0
+    assert wl.describe_nvfp4_plan(1, 16384, [(300, 512)])["ring"] == 0        # rank > 256
+    assert wl.describe_nvfp4_plan(1, 16384, [(300, 16, 2)])["ring"] == 0      # scales at +2 bytes
+    assert wl.describe_nvfp4_plan(1, 16384, [(300, 16)])["ring"] == 1
+    blocks = wl.describe_nvfp4_plan(1, 1152, [(300, 16)])
+    assert blocks["grid"] == (300 + 15) // 16
+    tiny = wl.describe_nvfp4_plan(1, 16384, [(16, 24)])
+    assert tiny["ring"] == 1 and tiny["grid"] == tiny["units"] == 8 + 1

@@ -43,11 +43,12 @@ def test_materialize_elementwise(N, K, r):
 
 
 def test_materialize_gemma3_mlp_shape():
-    """Gemma-3 1B gate shape (6912 x 1152) at rank 64; U V^T rows checked in full."""
-    p = wl_inputs.random_case(411, 1, 6912, 1152, 64).projs[0]
+    """The Gemma-3-1B gate shape of the decode workloads (4096 x 1152) at rank
+    64; 96 rows of W_eff checked in full."""
+    p = wl_inputs.random_case(411, 1, 4096, 1152, 64).projs[0]
     got = wl.materialize_weight(p.W0.cuda(), p.s.cuda(), p.U.cuda(), p.V.cuda())
     torch.cuda.synchronize()
-    rows = np.random.default_rng(5).choice(6912, 96, replace=False)
+    rows = np.random.default_rng(5).choice(4096, 96, replace=False)
     ref = (p.s.double().numpy()[rows, None] * p.W0.double().numpy()[rows]
            + p.U.double().numpy()[rows] @ p.V.double().numpy().T)
     g = got.double().cpu().numpy()[rows]

@@ -81,3 +81,43 @@ def test_short_wait_limit_gives_up_or_is_correct(path, case, mode, must_expire):
     # gave up left behind, the same call and a second one are correct
     check_call(call, path)
     check_call(wl_inputs.random_case(401 + M + N, M, N, K, r), path)
+
+
+def test_nvfp4_ring_short_wait_limit_gives_up_or_is_correct():
+    """The NVFP4 ring stream's slot waits (consumers on landed copies, the
+    producer on freed slots) at a 1 ns limit: each call gives up or is
+    correct; blocks split between CTAs leave their counters set when a call
+    gives up, which the status read clears, and the next call is correct."""
+    from oracle import nvfp4
+
+    M, Ns, K, rs = 2, [700, 2000], 16384, [256, 8]
+    assert wl.describe_nvfp4_plan(M, K, list(zip(Ns, rs)))["ring"] == 1
+    host, projs = [], []
+    for i, (N, r) in enumerate(zip(Ns, rs)):
+        codes, scales, ts = wl_inputs.draw_w0_nvfp4("fp4timeout", 1, 0, "all", f"f{i}", N, K)
+        s, U, V = wl_inputs.draw_delta("fp4timeout", 1, i, f"f{i}", N, K, r)
+        host.append((codes, scales, ts, s, U, V))
+        projs.append((codes.cuda(), scales.cuda(), ts, s.cuda(), U.cuda(), V.cuda()))
+    x = wl_inputs.draw_x("fp4timeout", 1, M, K)
+    refs = [nvfp4.forward(x, c.numpy(), sc.numpy(), ts, s, U, V) for (c, sc, ts, s, U, V) in host]
+    xd = x.cuda()
+    wl.set_wait_limit(1)
+    seen = []
+    try:
+        for _ in range(20):
+            ys = [torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda") for N in Ns]
+            wl.stacked_forward_nvfp4(xd, projs, ys=ys)
+            st = wl.last_device_status()
+            assert st in (0, TIMEOUT), st
+            seen.append(st)
+            if st == 0:
+                for y, ref in zip(ys, refs):
+                    compare(y.double().cpu().numpy(), ref, "nvfp4 ring under a 1 ns wait limit")
+    finally:
+        wl.set_wait_limit(0)
+    assert wl.last_device_status() == 0
+    for _ in range(2):
+        ys = wl.stacked_forward_nvfp4(xd, projs)
+        assert wl.last_device_status() == 0
+        for y, ref in zip(ys, refs):
+            compare(y.double().cpu().numpy(), ref, "nvfp4 ring after the time-outs")
