@@ -545,7 +545,8 @@ def nvfp4_figures(wl, peaks, seconds):
             "us_per_call": round(ms * 1e3, 2), "us_p10": round(per["p10_ms"] * 1e3, 2),
             "us_p90": round(per["p90_ms"] * 1e3, 2), "bytes_read_per_call": read,
             "bf16_path_weight_bytes_per_call": bf16, "bytes_ratio_vs_bf16": round(read / bf16, 4),
-            "launches_per_call": 2}
+            "launches_per_call": 2,
+            "stream": "ring" if wl.describe_nvfp4_plan(1, K, [(N, r) for N in Ns])["ring"] else "block"}
         del g, dev, outs
         torch.cuda.empty_cache()
     return out
