@@ -301,10 +301,14 @@ def build_workload(name):
 
 # --------------------------------------------------------------- roofline --
 ROOFLINE_CALLS = {
-    # name: (N per projection, K, r, M, label)
-    "gemma3_gate_up": (4096, 1152, 16, 1, "stacked gate/up decode, 2 x 4096 x 1152, r=16, M=1"),
-    "gemma4_gate_up": (21504, 5376, 256, 1, "stacked gate/up decode, 2 x 21504 x 5376, r=256, M=1"),
-    "gemma4_gate_up_m16": (21504, 5376, 256, 16, "stacked gate/up decode, 2 x 21504 x 5376, r=256, M=16"),
+    # name: (N of each projection, K, r, M, label)
+    "gemma3_gate_up": ([4096, 4096], 1152, 16, 1, "stacked gate/up decode, 2 x 4096 x 1152, r=16, M=1"),
+    "gemma3_qkv": ([1024, 256, 256], 1152, 16, 1, "stacked q/k/v decode, (1024 + 256 + 256) x 1152, r=16, M=1"),
+    "gemma3_o": ([1152], 1024, 16, 1, "o decode, 1152 x 1024, r=16, M=1"),
+    "gemma3_down": ([1152], 4096, 16, 1, "down decode, 1152 x 4096, r=16, M=1"),
+    "gemma4_gate_up": ([21504, 21504], 5376, 256, 1, "stacked gate/up decode, 2 x 21504 x 5376, r=256, M=1"),
+    "gemma4_gate_up_m16": ([21504, 21504], 5376, 256, 16,
+                           "stacked gate/up decode, 2 x 21504 x 5376, r=256, M=16"),
 }
 
 
@@ -313,20 +317,19 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     calls that rotate through enough distinct bundles (> 3x L2) that every
     launch streams its weights from HBM.  The default is the dominant kernel
     of the Gemma-3-1B decode step: the stacked gate/up call."""
-    N, K, r, M, label = ROOFLINE_CALLS[call]
-    call_bytes = 2 * footprint.call_weight_bytes(N, K, r) + footprint.call_io_bytes(M, 2 * N, K)
-    copies = max(4, (3 * L2_BYTES) // (2 * N * K * 2) + 1)
+    Ns, K, r, M, label = ROOFLINE_CALLS[call]
+    call_bytes = sum(footprint.call_weight_bytes(N, K, r) for N in Ns) + footprint.call_io_bytes(M, sum(Ns), K)
+    copies = max(4, (3 * L2_BYTES) // (sum(Ns) * K * 2) + 1)
     calls = []
     for i in range(copies):
-        c = wl_inputs.random_case(1000 + i, M, [N, N], K, [r, r], P=2)
+        c = wl_inputs.random_case(1000 + i, M, list(Ns), K, [r] * len(Ns), P=len(Ns))
         calls.append(to_dev_call(c))
-    outs = [[torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-            for _ in calls]
+    outs = [[torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for N in Ns] for _ in calls]
     g = capture(make_step(calls, outs, wl), 3)
     st = per_call(time_windows(g, seconds), copies)
     ms = st["median_ms"]
     achieved = call_bytes / (ms * 1e-3) / 1e9
-    path = call_path(M, [(N, r), (N, r)], K)
+    path = call_path(M, [(N, r) for N in Ns], K)
     kernel = {"rows": "rows_kernel", "decode": "decode_kernel"}.get(path, "gemm_kernel")
     traffic = traffic_from_profile(kernel, call)
     return {"kernel": f"{kernel} (one launch per call: W0 x, V^T x and the epilogue fused)",
@@ -384,7 +387,13 @@ def sweep_roofline(wl, peaks, calls, dev_calls, outs, seconds):
     ft = sum(per[f]["us"] for f in groups[dom])
     achieved = fb / (ft * 1e-6) / 1e9
     kernel = f"rows_kernel<{dom[0]}, {dom[1]}, {dom[2]}>" if dom else "decode_kernel"
-    traffic = traffic_from_profile("rows_kernel", "gemma3_gate_up") if dom == (1, 4, 1) else None
+    traffic = None
+    if dom == (1, 4, 1) and groups[dom] == ["gate+up"]:
+        traffic = traffic_from_profile("rows_kernel", "gemma3_gate_up")
+    elif sorted(groups[dom]) == ["down", "o", "q+k+v"]:
+        # the group's bytes are one call of each family: so is its traffic
+        parts = [traffic_from_profile("rows_kernel", f"gemma3_{c}") for c in ("qkv", "o", "down")]
+        traffic = sum(parts) if all(t is not None for t in parts) else None
     return {"kernel": kernel + " (one launch per call: W0 x, V^T x, U T and the epilogue fused)",
             "calls": "+".join(groups[dom]), "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -510,16 +519,19 @@ def secondary_figures(wl, peaks, headline_ms, seconds):
     return out
 
 
-def nvfp4_figures(wl, peaks, seconds):
+NVFP4_FAMILIES = {"qkv_sliding": ([8192, 4096, 4096], 5376), "o_sliding": ([5376], 8192),
+                  "qk_full": ([16384, 2048], 5376), "o_full": ([5376], 16384),
+                  "gate_up": ([21504, 21504], 5376), "down": ([5376], 21504)}
+
+
+def nvfp4_figures(wl, peaks, seconds, only=None):
     """The NVFP4 decode path on the Gemma-4-31B decode families at M = 1
     (rank 256, three distinct bundles per family, rotating): GB/s of the bytes
     the call reads (codes, block scales, s, U, V), and the weight bytes per
     token against the bf16 path's."""
     from linear_wl_forward_b200 import footprint as fpt
 
-    fams = {"qkv_sliding": ([8192, 4096, 4096], 5376), "o_sliding": ([5376], 8192),
-            "qk_full": ([16384, 2048], 5376), "o_full": ([5376], 16384),
-            "gate_up": ([21504, 21504], 5376), "down": ([5376], 21504)}
+    fams = {k: v for k, v in NVFP4_FAMILIES.items() if only is None or k == only}
     out = {}
     r = 256
     for name, (Ns, K) in fams.items():
@@ -722,6 +734,8 @@ def main():
                     help="time only the dominant kernel's call (the command the ncu summaries profile)")
     ap.add_argument("--call", default="gemma3_gate_up", choices=sorted(ROOFLINE_CALLS),
                     help="the call --roofline-only times")
+    ap.add_argument("--nvfp4-only", default=None, choices=sorted(NVFP4_FAMILIES),
+                    help="time only this Gemma-4-31B family on the NVFP4 path (the command the NVFP4 ncu summaries profile)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the Gemma-4-31B gate/up prefill call (the command the GEMM ncu summary profiles)")
     args = ap.parse_args()
@@ -746,6 +760,9 @@ def main():
 
     wl.lib()  # fails loudly if the CUDA library is missing
     peaks = load_peaks()
+    if args.nvfp4_only:
+        print(json.dumps({"nvfp4": nvfp4_figures(wl, peaks, args.seconds, args.nvfp4_only)}), flush=True)
+        return
     if args.roofline_only:
         print(json.dumps({"roofline": decode_roofline(wl, peaks, args.call, args.seconds)}), flush=True)
         return
