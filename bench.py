@@ -148,10 +148,13 @@ def to_dev_call(call):
 
 def call_path(M, projs_nr, K=None):
     """The kernel path the library's automatic choice takes for a call
-    (wl_path in include/wl.h): 'rows', 'decode' or 'gemm'."""
+    (wl_path in include/wl.h): 'ring', 'rows', 'decode' or 'gemm'."""
     import linear_wl_forward_b200 as wl
 
     rows = sum(n for n, _ in projs_nr)
+    if (K is not None and M <= 8 and 2 * rows * K >= (64 << 20) and not (M >= 5 and rows >= 32768)
+            and all(r % 8 == 0 and r <= 256 for _, r in projs_nr)):
+        return "ring"
     if M <= 4 or (M <= wl.DECODE_MAX_M and rows < 8192):
         if K is not None:
             try:
@@ -167,6 +170,8 @@ def launches_per_call(path, ranks):
     """Kernels one call launches (the library's own kernels)."""
     if path in ("rows", "decode"):
         return 1  # one fused kernel: W0 x, V^T x and the epilogue
+    if path == "ring":
+        return 2  # V^T x and the permuted x, then the weight stream
     n = 1
     if any(ranks):
         n += 2  # one V transpose for all projections + the T = x V GEMM
@@ -330,7 +335,7 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     ms = st["median_ms"]
     achieved = call_bytes / (ms * 1e-3) / 1e9
     path = call_path(M, [(N, r) for N in Ns], K)
-    kernel = {"rows": "rows_kernel", "decode": "decode_kernel"}.get(path, "gemm_kernel")
+    kernel = {"rows": "rows_kernel", "decode": "decode_kernel", "ring": "ring_kernel<true>"}.get(path, "gemm_kernel")
     traffic = traffic_from_profile(kernel, call)
     return {"kernel": f"{kernel} (one launch per call: W0 x, V^T x and the epilogue fused)",
             "call": label, "path": path,

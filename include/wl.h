@@ -86,9 +86,12 @@ typedef struct {
     int r;             /* rank of the delta, 0 <= r <= WL_MAX_RANK     */
 } wl_proj;
 
-/* Which kernels a forward call uses.  WL_PATH_AUTO takes a decode kernel for
- * M <= 4, and for M <= WL_DECODE_MAX_M when the call's projections total fewer
- * than 8192 output rows; otherwise the tensor-core GEMM.  Of the two decode
+/* Which kernels a forward call uses.  WL_PATH_AUTO takes the persistent ring
+ * for calls of at most 8 tokens whose weights total at least 64 MB (except
+ * 5-8 tokens over 32768 or more output rows) when the call fits it; else a
+ * decode kernel for M <= 4, and for M <= WL_DECODE_MAX_M when the call's
+ * projections total fewer than 8192 output rows; otherwise the tensor-core
+ * GEMM.  Of the two decode
  * kernels it takes the row-stream one whenever the call fits it (short calls:
  * at most four 16-row blocks of W0 per SM, every rank <= 64 and a multiple of
  * 8, U and V 16-byte aligned), else the weight-streaming one.  The others
@@ -97,8 +100,12 @@ typedef enum {
     WL_PATH_AUTO = 0,
     WL_PATH_DECODE = 1, /* weight-streaming kernel (bulk copies + warp MMA), 1 <= M <= WL_DECODE_MAX_M */
     WL_PATH_GEMM = 2,   /* tcgen05 tensor-core GEMM with the fused low-rank epilogue */
-    WL_PATH_ROWS = 3    /* row-stream decode kernel (register-fed warp MMA, K split over CTA
+    WL_PATH_ROWS = 3,   /* row-stream decode kernel (register-fed warp MMA, K split over CTA
                            clusters) for short calls; WL_ERR_UNSUPPORTED for calls it does not fit */
+    WL_PATH_RING = 4    /* persistent ring decode (a V^T x launch, then one CTA per SM streaming
+                           16-row x 512-column weight tiles by TMA, the call's work split evenly
+                           over the SMs) for 1 <= M <= 8, ranks <= 256 and multiples of 8, U, V
+                           and s 16-byte aligned; WL_ERR_UNSUPPORTED otherwise */
 } wl_path;
 
 #define WL_DECODE_MAX_M 16

@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libwl.so")
 
 STATUS = {0: "WL_OK", 1: "WL_ERR_INVALID_ARG", 2: "WL_ERR_ALIGNMENT", 3: "WL_ERR_UNSUPPORTED",
           4: "WL_ERR_CUDA", 5: "WL_ERR_TIMEOUT", 6: "WL_ERR_NOMEM", 7: "WL_ERR_NOT_CONVERGED"}
-PATHS = {"auto": 0, "decode": 1, "gemm": 2, "rows": 3}
+PATHS = {"auto": 0, "decode": 1, "gemm": 2, "rows": 3, "ring": 4}
 DECODE_MAX_M = 16
 MAX_RANK = 1024
 MAX_PROJ = 8

@@ -192,7 +192,8 @@ wl_status validate(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, 
     if (!projs) return WL_ERR_INVALID_ARG;
     if (P < 1 || P > WL_MAX_PROJ) return P < 1 ? WL_ERR_INVALID_ARG : WL_ERR_UNSUPPORTED;
     if (M < 0 || K < 0) return WL_ERR_INVALID_ARG;
-    if (path != WL_PATH_AUTO && path != WL_PATH_DECODE && path != WL_PATH_GEMM && path != WL_PATH_ROWS)
+    if (path != WL_PATH_AUTO && path != WL_PATH_DECODE && path != WL_PATH_GEMM && path != WL_PATH_ROWS &&
+        path != WL_PATH_RING)
         return WL_ERR_INVALID_ARG;
     for (int i = 0; i < P; ++i) {
         const wl_proj &q = projs[i];
@@ -245,6 +246,20 @@ wl_status build_prefetch(const wl_range *ranges, int n, PrefetchList &pf) {
 //   stacked gate/up 2 x 4096 x 1152, M = 8: GEMM 26.9 us, decode 30.1 us
 //   down 5376 x 21504, M = 8 / 16: decode 107 / 141 us, GEMM 231 / 234 us
 //   q/k/v 1536 x 1152, M = 8: decode 19.5 us, GEMM 22.9 us
+// Large calls of at most 8 tokens take the persistent ring: at least 64 MB
+// of bf16 weights (the Gemma-4-31B projections; measured against the other
+// kernels: q/k/v 57 against 66 us at M = 1, down 68 against 129 us at M = 2,
+// o 56 against 145 us at M = 8), except wide calls of 5-8 tokens over 32768 or
+// more rows, where the tensor-core GEMM is faster (gate/up 136 against 155 us
+// at M = 8).
+bool auto_ring(int M, int K, const wl_proj *projs, int P) {
+    if (M > kFp4MaxM) return false;
+    long long rows = 0;
+    for (int i = 0; i < P; ++i) rows += projs[i].N;
+    if (2LL * rows * K < (64LL << 20)) return false;
+    return !(M >= 5 && rows >= 32768);
+}
+
 bool auto_decode(int M, const wl_proj *projs, int P) {
     if (M > WL_DECODE_MAX_M) return false;
     if (M <= 4) return true;
@@ -554,6 +569,84 @@ wl_status run_gemm(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_pr
     return from_cuda(launch_gemm(gp, pool.num_sms, stream));
 }
 
+// Scratch and launch of a planned NVFP4 (or bf16-ring) call; g_mu held.
+wl_status fp4_run(DevicePool &pool, Fp4Params &fp, cudaStream_t stream) {
+    wl_status st;
+    const int M = fp.M;
+    const size_t tl = (size_t)(fp.t_ld > 0 ? fp.t_ld : 1);
+    void *xq = nullptr, *tp = nullptr, *gp = nullptr, *tt = nullptr, *cnt = nullptr;
+    if ((st = scratch(pool, kSlotXh, fp4_xq_halves(fp) * 2, &xq)) != WL_OK) return st;
+    if ((st = scratch(pool, kSlotFp4Part, (size_t)fp.slices * M * tl * sizeof(float), &tp)) != WL_OK) return st;
+    if ((st = scratch(pool, kSlotFp4G, (size_t)fp.ngrp * M * tl * sizeof(float), &gp)) != WL_OK) return st;
+    if ((st = scratch(pool, kSlotFp4T, (size_t)M * tl * sizeof(float), &tt)) != WL_OK) return st;
+    if ((st = scratch(pool, kSlotFp4Cnt, (size_t)(kMaxSeg * (fp.ngrp + 1)) * sizeof(unsigned), &cnt, true)) != WL_OK)
+        return st;
+    fp.xq = static_cast<__half *>(xq);
+    fp.Tpart = static_cast<float *>(tp);
+    fp.Gpart = static_cast<float *>(gp);
+    fp.T = static_cast<float *>(tt);
+    fp.cnt = static_cast<unsigned int *>(cnt);
+    if (fp.ring) {
+        void *pa = nullptr, *bc = nullptr;
+        if ((st = scratch(pool, kSlotFp4Blk, (size_t)fp.grid * 2 * 16 * kFp4MaxM * sizeof(float2), &pa)) != WL_OK)
+            return st;
+        if ((st = scratch(pool, kSlotFp4BCnt, (size_t)fp.total_blocks * sizeof(unsigned), &bc, true)) != WL_OK)
+            return st;
+        fp.parts = static_cast<float2 *>(pa);
+        fp.bcnt = static_cast<unsigned int *>(bc);
+    }
+    return from_cuda(launch_fp4(fp, stream));
+}
+
+// The bf16 forward on the persistent ring (prep launch for V^T x and the
+// permuted x, then the ring): WL_ERR_UNSUPPORTED for calls it does not take.
+wl_status ring_params(Fp4Params &fp, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, int num_sms,
+                      bool encode_maps) {
+    if (M < 1 || M > kFp4MaxM) return WL_ERR_UNSUPPORTED;
+    std::memset(&fp, 0, sizeof fp);
+    int blocks = 0, t_off = 0, nr = 0;
+    for (int i = 0; i < P; ++i) {
+        const wl_proj &q = projs[i];
+        if (q.N == 0) continue;
+        if (q.r % 8 != 0 || q.r > kFp4RingMaxRank) return WL_ERR_UNSUPPORTED;
+        if (q.r > 0 && (!aligned16(q.U) || !aligned16(q.V))) return WL_ERR_UNSUPPORTED;
+        Fp4Seg &sg = fp.seg[fp.nseg++];
+        sg.codes = reinterpret_cast<const uint8_t *>(q.W0);
+        sg.scales = nullptr;
+        sg.ts = 1.f;
+        sg.s = q.s;
+        sg.U = reinterpret_cast<const __nv_bfloat16 *>(q.U);
+        sg.V = reinterpret_cast<const __nv_bfloat16 *>(q.V);
+        sg.y = reinterpret_cast<__nv_bfloat16 *>(q.y);
+        sg.N = q.N;
+        sg.r = q.r;
+        sg.blk_begin = blocks;
+        sg.t_off = t_off;
+        blocks += (q.N + 15) / 16;
+        t_off += q.r;
+        nr += q.r > 0;
+    }
+    if (fp.nseg == 0) return WL_ERR_UNSUPPORTED;
+    fp.bf16 = 1;
+    fp.M = M;
+    fp.K = K;
+    fp.total_blocks = blocks;
+    fp.t_ld = t_off;
+    fp.nr = nr;
+    fp.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    return plan_fp4(fp, num_sms, encode_maps);
+}
+
+wl_status run_ring(DevicePool &pool, const wl_bf16 *x, int M, int K, const wl_proj *projs, int P,
+                   cudaStream_t stream) {
+    static Fp4Params fp;  // guarded by g_mu
+    wl_status st = ring_params(fp, x, M, K, projs, P, pool.num_sms, true);
+    if (st != WL_OK) return st;
+    fp.status = pool.words;
+    fp.timeout_ns = wait_limit_ns();
+    return fp4_run(pool, fp, stream);
+}
+
 wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, wl_path path,
                   const wl_range *prefetch, int nprefetch, void *stream_ptr) {
     wl_status st = validate(x, M, K, projs, P, path);
@@ -574,6 +667,10 @@ wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, w
     std::lock_guard<std::mutex> lock(g_mu);
     DevicePool *pool = nullptr;
     if ((st = pool_for_current_device(&pool)) != WL_OK) return st;
+    if (path == WL_PATH_AUTO && auto_ring(M, K, projs, P)) {
+        st = run_ring(*pool, x, M, K, projs, P, stream);
+        if (st != WL_ERR_UNSUPPORTED) return st;
+    }
     if (path == WL_PATH_AUTO && auto_decode(M, projs, P)) {
         // Each decode kernel declines shapes it cannot hold (before launching
         // anything): short calls take the row-stream kernel, the rest the
@@ -584,6 +681,7 @@ wl_status forward(const wl_bf16 *x, int M, int K, const wl_proj *projs, int P, w
         return st == WL_ERR_UNSUPPORTED ? run_gemm(*pool, x, M, K, projs, P, pf, stream) : st;
     }
     if (path == WL_PATH_ROWS) return run_rows(*pool, x, M, K, projs, P, pf, stream);
+    if (path == WL_PATH_RING) return run_ring(*pool, x, M, K, projs, P, stream);
     return path == WL_PATH_DECODE ? run_decode(*pool, x, M, K, projs, P, pf, stream)
                                   : run_gemm(*pool, x, M, K, projs, P, pf, stream);
 }
@@ -787,30 +885,7 @@ wl_status wl_stacked_forward_nvfp4(const wl_bf16 *x, int M, int K, const wl_proj
     fp.status = pool->words;
     fp.timeout_ns = wait_limit_ns();
     if ((st = plan_fp4(fp, pool->num_sms)) != WL_OK) return st;
-    const size_t tl = (size_t)(fp.t_ld > 0 ? fp.t_ld : 1);
-    void *xq = nullptr, *tp = nullptr, *gp = nullptr, *tt = nullptr, *cnt = nullptr;
-    if ((st = scratch(*pool, kSlotXh, fp4_xq_halves(fp) * 2, &xq)) != WL_OK) return st;
-    if ((st = scratch(*pool, kSlotFp4Part, (size_t)fp.slices * M * tl * sizeof(float), &tp)) != WL_OK) return st;
-    if ((st = scratch(*pool, kSlotFp4G, (size_t)fp.ngrp * M * tl * sizeof(float), &gp)) != WL_OK) return st;
-    if ((st = scratch(*pool, kSlotFp4T, (size_t)M * tl * sizeof(float), &tt)) != WL_OK) return st;
-    if ((st = scratch(*pool, kSlotFp4Cnt, (size_t)(kMaxSeg * (fp.ngrp + 1)) * sizeof(unsigned), &cnt, true)) !=
-        WL_OK)
-        return st;
-    fp.xq = static_cast<__half *>(xq);
-    fp.Tpart = static_cast<float *>(tp);
-    fp.Gpart = static_cast<float *>(gp);
-    fp.T = static_cast<float *>(tt);
-    fp.cnt = static_cast<unsigned int *>(cnt);
-    if (fp.ring) {
-        void *pa = nullptr, *bc = nullptr;
-        if ((st = scratch(*pool, kSlotFp4Blk, (size_t)fp.grid * 2 * 16 * kFp4MaxM * sizeof(float2), &pa)) != WL_OK)
-            return st;
-        if ((st = scratch(*pool, kSlotFp4BCnt, (size_t)fp.total_blocks * sizeof(unsigned), &bc, true)) != WL_OK)
-            return st;
-        fp.parts = static_cast<float2 *>(pa);
-        fp.bcnt = static_cast<unsigned int *>(bc);
-    }
-    return from_cuda(launch_fp4(fp, stream));
+    return fp4_run(*pool, fp, stream);
 }
 
 wl_status wl_describe_nvfp4_plan(int M, int K, const wl_proj_nvfp4 *projs, int P, int num_sms,

@@ -239,6 +239,7 @@ struct Fp4Params {
     float *T;             // [M][t_ld]
     unsigned int *cnt;    // [nr][ngrp] group counters, then [nr] projection counters (zeroed, self-resetting)
     // ring
+    int bf16;             // 1: W0 in bf16 (codes = the bf16 rows, no scales, tensor scale 1); ring stream only
     int ring;             // 1: ring stream, 0: block stream
     int grid, ns, slot_bytes, smem, nst;
     long long utot;

@@ -209,6 +209,13 @@ __device__ __forceinline__ size_t xq_index(int m, int k, int Mp) {
     return ((((size_t)kg * 4 + t) * Mp + m) * 4 + q) * 8 + j;
 }
 
+// Index of x[m][k] in the permuted bf16 copy of the bf16-weight ring: per
+// 32-column group, lane q's eight consecutive columns 8q .. 8q + 7, tokens
+// (Mp of them) in between: [k / 32][m][q][8].
+__device__ __forceinline__ size_t xb_index(int m, int k, int Mp) {
+    return ((((size_t)(k >> 5) * Mp + m) * 4 + ((k >> 3) & 3)) * 8) + (k & 7);
+}
+
 // The pj-th projection with a delta (-1 if none).
 __device__ __forceinline__ int delta_seg(const Fp4Params &P, int pj) {
     for (int i = 0, n = 0; i < P.nseg; ++i)
@@ -235,9 +242,23 @@ __global__ void __launch_bounds__(kPrepThreads) fp4_prep_kernel(const __grid_con
     const int k0 = sl * kr, k1 = min(K, k0 + kr), nk = k1 - k0;
     for (int i = tid; i < Mp * nk; i += kPrepThreads) {
         const int m = i / nk, k = k0 + i - m * nk;
-        const float v = m < M ? __bfloat162float(P.x[(size_t)m * K + k]) : 0.f;
+        const __nv_bfloat16 xb = m < M ? P.x[(size_t)m * K + k] : __float2bfloat16_rn(0.f);
+        const float v = __bfloat162float(xb);
         if (m < M) xs[m * kr + (k - k0)] = v;
-        if (pj == 0) P.xq[xq_index(m, k, Mp)] = __float2half_rn(v);
+        if (pj == 0) {
+            if (P.bf16)
+                reinterpret_cast<__nv_bfloat16 *>(P.xq)[xb_index(m, k, Mp)] = xb;
+            else
+                P.xq[xq_index(m, k, Mp)] = __float2half_rn(v);
+        }
+    }
+    if (P.bf16 && pj == 0 && k1 == K) {
+        // the last 32-column group's columns past K are zero
+        const int kp = (K + 31) & ~31;
+        for (int i = tid; i < Mp * (kp - K); i += kPrepThreads) {
+            const int m = i / (kp - K), k = K + i - m * (kp - K);
+            reinterpret_cast<__nv_bfloat16 *>(P.xq)[xb_index(m, k, Mp)] = __float2bfloat16_rn(0.f);
+        }
     }
     __syncthreads();
     const int sp = delta_seg(P, pj);
@@ -503,7 +524,8 @@ __device__ __forceinline__ int cta_of(long long utot, int G, long long u) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kRingThreads, 1) fp4_ring_kernel(const __grid_constant__ Fp4Params P) {
+template <bool BF16>
+__global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_constant__ Fp4Params P) {
     pdl_launch_dependents();
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -519,14 +541,18 @@ __global__ void __launch_bounds__(kRingThreads, 1) fp4_ring_kernel(const __grid_
     const int G = gridDim.x, c = blockIdx.x;
     const long long utot = P.utot;
     const long long u0 = range_start(utot, G, c), u1 = range_start(utot, G, c + 1);
-    const int K = P.K, M = P.M, Mp = P.Mp, nkg = K / FKG, nst = P.nst;
-    const uint32_t xstage = 256u * (uint32_t)Mp;  // bytes of permuted x per k-group
-    const uint32_t sv_off = kCodeBytes + kScaleBytes + (uint32_t)kFp4StageKG * xstage;  // 16 row scales
+    // k-units: 128-column k-groups of NVFP4 codes, or 32-column groups of
+    // bf16 weights; a stage holds kFp4StageKG of them (1 KB of each row)
+    constexpr uint32_t SCB = BF16 ? 0u : kScaleBytes;  // block scales of a stage
+    const int K = P.K, M = P.M, Mp = P.Mp, nst = P.nst;
+    const int nkg = BF16 ? (K + 31) / 32 : K / FKG;
+    const uint32_t xstage = (BF16 ? 64u : 256u) * (uint32_t)Mp;  // bytes of permuted x per k-unit
+    const uint32_t sv_off = kCodeBytes + SCB + (uint32_t)kFp4StageKG * xstage;  // 16 row scales
 
     if (warp == FW && lane < P.nseg) {
         // the tensor maps into the descriptor cache before the first copy
         prefetch_tmap(&P.tm_c[lane]);
-        prefetch_tmap(&P.tm_s[lane]);
+        if (!BF16) prefetch_tmap(&P.tm_s[lane]);
         prefetch_tmap(&P.tm_sv[lane]);
         if (P.seg[lane].r > 0) prefetch_tmap(&P.tm_u[lane]);
     }
@@ -559,7 +585,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) fp4_ring_kernel(const __grid_
             auto issue_dep = [&](int sl, const UnitCursor &c) {
                 if (c.st < nst) {
                     const int kgs = min(kFp4StageKG, nkg - kFp4StageKG * c.st);
-                    bulk_load(ring + (size_t)sl * SB + kCodeBytes + kScaleBytes,
+                    bulk_load(ring + (size_t)sl * SB + kCodeBytes + SCB,
                               reinterpret_cast<const uint8_t *>(P.xq) + (size_t)kFp4StageKG * c.st * xstage,
                               (uint32_t)kgs * xstage, &full[sl]);
                 } else {
@@ -596,9 +622,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) fp4_ring_kernel(const __grid_
                 const uint32_t sbytes = first ? 64u : 0u;
                 if (cu.st < nst) {
                     const int kgs = min(kFp4StageKG, nkg - kFp4StageKG * cu.st);
-                    mbar_arrive_expect_tx(&full[slot], kCodeBytes + kScaleBytes + (uint32_t)kgs * xstage + sbytes);
+                    mbar_arrive_expect_tx(&full[slot], kCodeBytes + SCB + (uint32_t)kgs * xstage + sbytes);
                     tma_2d(sb, &P.tm_c[cu.sp], (int)(kCodeBytes / 64) * cu.st, row0, &full[slot], pol);
-                    tma_2d(sb + kCodeBytes, &P.tm_s[cu.sp], (int)(kScaleBytes / 64) * cu.st, row0, &full[slot], pol);
+                    if (!BF16)
+                        tma_2d(sb + kCodeBytes, &P.tm_s[cu.sp], (int)(kScaleBytes / 64) * cu.st, row0, &full[slot], pol);
                 } else {
                     mbar_arrive_expect_tx(&full[slot], 32u * (uint32_t)S.r + 4u * (uint32_t)(M * S.r) + sbytes);
                     tma_2d(sb, &P.tm_u[cu.sp], 0, row0, &full[slot], pol);
@@ -653,11 +680,24 @@ __global__ void __launch_bounds__(kRingThreads, 1) fp4_ring_kernel(const __grid_
                         const int kgl = warp + FW * j;
                         if (kFp4StageKG * cu.st + kgl >= nkg) break;
                         const uint32_t cb = sa + 64u * kgl + 16u * q;
+                        if (BF16) {
+                            // 32 columns of rows g and g + 8: the lane's eight
+                            // (8q .. 8q + 7) are the logical columns 2q, 2q + 1,
+                            // 2q + 8, 2q + 9 of two MMAs, as in x's copy
+                            const uint4 w0 = lds128(cb + g * (kCodeBytes / 16)), w1 = lds128(cb + (g + 8) * (kCodeBytes / 16));
+                            const uint4 bx = xv ? lds128(sa + kCodeBytes + (uint32_t)(((kgl * Mp + g) * 4 + q) * 16))
+                                                : make_uint4(0u, 0u, 0u, 0u);
+                            const uint32_t a1[4] = {w0.x, w1.x, w0.y, w1.y};
+                            const uint32_t a2[4] = {w0.z, w1.z, w0.w, w1.w};
+                            mma_bf16(acc[(2 * j) & 3], a1, bx.x, bx.y);
+                            mma_bf16(acc[(2 * j + 1) & 3], a2, bx.z, bx.w);
+                            continue;
+                        }
                         const uint4 c0 = lds128(cb + g * (kCodeBytes / 16)), c1 = lds128(cb + (g + 8) * (kCodeBytes / 16));
                         const uint32_t sbs = sa + kCodeBytes + 8u * kgl + 2u * q;
                         const uint16_t s0 = lds16(sbs + g * (kScaleBytes / 16)), s1 = lds16(sbs + (g + 8) * (kScaleBytes / 16));
                         uint4 xf[4];
-                        const uint32_t xb = sa + kCodeBytes + kScaleBytes;
+                        const uint32_t xb = sa + kCodeBytes + SCB;
 #pragma unroll
                         for (int t = 0; t < 4; ++t)
                             xf[t] = xv ? lds128(xb + (uint32_t)((((kgl * 4 + t) * Mp + g) * 4 + q) * 16))
@@ -786,7 +826,9 @@ namespace {
 std::atomic<bool> g_ring_attr{false};
 }
 
-size_t fp4_xq_halves(const Fp4Params &p) { return (size_t)(p.K / FKG) * 4 * p.Mp * 4 * 8; }
+size_t fp4_xq_halves(const Fp4Params &p) {
+    return p.bf16 ? (size_t)((p.K + 31) / 32) * 32 * p.Mp : (size_t)(p.K / FKG) * 4 * p.Mp * 4 * 8;
+}
 
 wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     const int K = p.K, M = p.M;
@@ -801,20 +843,21 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     p.kr = kr;
     p.slices = (K + kr - 1) / kr;
     p.ngrp = (p.slices + kFp4GroupSlices - 1) / kFp4GroupSlices;
-    // ring stream when the scale rows are 16-byte strided and every rank fits one U unit
-    bool ring = K % 256 == 0;
+    // ring stream when every rank fits one U unit, s is 16-byte aligned (its
+    // TMA box) and, for NVFP4, the scale rows are 16-byte strided
+    bool ring = p.bf16 ? true : K % 256 == 0;
     for (int i = 0; i < p.nseg; ++i)
-        ring = ring && p.seg[i].r <= kFp4RingMaxRank && (reinterpret_cast<uintptr_t>(p.seg[i].scales) & 15u) == 0 &&
-               (reinterpret_cast<uintptr_t>(p.seg[i].s) & 15u) == 0;
-    // ... and when the call has few row blocks per SM, each of a long K: the
-    // ring balances them evenly over the SMs.  Otherwise one CTA per block
-    // streams faster (measured on the Gemma-4-31B families: the ring wins
-    // only for down, 5376 x 21504; q 8192 x 5376 and o 5376 x 8192, also few
-    // blocks, run faster per block)
-    ring = ring && p.total_blocks <= kFp4RingMaxBlocksPerSm * num_sms && K >= kFp4RingMinK;
+        ring = ring && p.seg[i].r <= kFp4RingMaxRank && (reinterpret_cast<uintptr_t>(p.seg[i].s) & 15u) == 0 &&
+               (p.bf16 || (reinterpret_cast<uintptr_t>(p.seg[i].scales) & 15u) == 0);
+    // NVFP4: and when the call has few row blocks per SM, each of a long K:
+    // the ring balances them evenly over the SMs.  Otherwise one CTA per
+    // block streams faster (measured on the Gemma-4-31B families: the ring
+    // wins only for down, 5376 x 21504; q 8192 x 5376 and o 5376 x 8192, also
+    // few blocks, run faster per block).  bf16 weights: the caller decides.
+    if (!p.bf16) ring = ring && p.total_blocks <= kFp4RingMaxBlocksPerSm * num_sms && K >= kFp4RingMinK;
     p.ring = ring ? 1 : 0;
-    if (!ring) return WL_OK;
-    const int nkg = K / FKG;
+    if (!ring) return p.bf16 ? WL_ERR_UNSUPPORTED : WL_OK;
+    const int nkg = p.bf16 ? (K + 31) / 32 : K / FKG;  // k-units
     p.nst = (nkg + kFp4StageKG - 1) / kFp4StageKG;
     long long ub = 0;
     for (int i = 0; i < p.nseg; ++i) {
@@ -825,23 +868,29 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     }
     p.utot = ub;
     p.grid = (int)std::min<long long>(num_sms, ub);
-    const uint32_t slot = (kCodeBytes + kScaleBytes + (uint32_t)kFp4StageKG * 256u * p.Mp + 64u + 1023u) & ~1023u;
+    const uint32_t slot =
+        (kCodeBytes + (p.bf16 ? 0u : kScaleBytes) + (uint32_t)kFp4StageKG * (p.bf16 ? 64u : 256u) * p.Mp + 64u + 1023u) &
+        ~1023u;
     p.slot_bytes = (int)slot;
     const uint32_t fixed = 2u * FW * 32 * 2 * 16 + 32 + 1024;  // reduction buffers, flags, alignment
     int ns = (int)((kRingSmemMax - fixed) / (slot + 16));
     ns = std::min(ns, kFp4RingMaxStages);
     if (ns < kIssueLanes) {
         p.ring = 0;
-        return WL_OK;
+        return p.bf16 ? WL_ERR_UNSUPPORTED : WL_OK;
     }
     p.ns = ns;
     p.smem = (int)((uint32_t)ns * slot + 2u * FW * 32 * 2 * 16 + 16u * ns + 32 + 1024);
     for (int i = 0; encode_maps && i < p.nseg; ++i) {
         const Fp4Seg &sg = p.seg[i];
         wl_status st;
-        if ((st = encode_map_2d_u32(&p.tm_c[i], sg.codes, (uint64_t)K / 8, sg.N, (uint64_t)K / 2, kCodeBytes / 64, 16)) != WL_OK)
+        // the weight rows as 32-bit words (K/8 of them for NVFP4 codes, K/2 for bf16)
+        const uint64_t wwords = p.bf16 ? (uint64_t)K / 2 : (uint64_t)K / 8;
+        if ((st = encode_map_2d_u32(&p.tm_c[i], sg.codes, wwords, sg.N, wwords * 4, kCodeBytes / 64, 16)) != WL_OK)
             return st;
-        if ((st = encode_map_2d_u32(&p.tm_s[i], sg.scales, (uint64_t)K / 64, sg.N, (uint64_t)K / 16, kScaleBytes / 64, 16)) != WL_OK)
+        if (!p.bf16 &&
+            (st = encode_map_2d_u32(&p.tm_s[i], sg.scales, (uint64_t)K / 64, sg.N, (uint64_t)K / 16, kScaleBytes / 64, 16)) !=
+                WL_OK)
             return st;
         if (sg.r > 0 &&
             (st = encode_map_2d_u32(&p.tm_u[i], sg.U, (uint64_t)sg.r / 2, sg.N, (uint64_t)sg.r * 2, sg.r / 2, 16)) !=
@@ -866,14 +915,16 @@ cudaError_t launch_fp4(const Fp4Params &p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (p.ring) {
         if (!g_ring_attr.load(std::memory_order_acquire)) {
-            e = cudaFuncSetAttribute(fp4_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+            e = cudaFuncSetAttribute(ring_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(ring_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
             if (e != cudaSuccess) return e;
             g_ring_attr.store(true, std::memory_order_release);
         }
         cfg.blockDim = dim3(kRingThreads);
         cfg.gridDim = dim3((unsigned)p.grid);
         cfg.dynamicSmemBytes = (size_t)p.smem;
-        return cudaLaunchKernelEx(&cfg, fp4_ring_kernel, p);
+        return p.bf16 ? cudaLaunchKernelEx(&cfg, ring_kernel<true>, p) : cudaLaunchKernelEx(&cfg, ring_kernel<false>, p);
     }
     cfg.blockDim = dim3(FTH);
     cfg.gridDim = dim3((unsigned)p.total_blocks);
