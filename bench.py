@@ -337,7 +337,9 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     path = call_path(M, [(N, r) for N in Ns], K)
     kernel = {"rows": "rows_kernel", "decode": "decode_kernel", "ring": "ring_kernel<true>"}.get(path, "gemm_kernel")
     traffic = traffic_from_profile(kernel, call)
-    return {"kernel": f"{kernel} (one launch per call: W0 x, V^T x and the epilogue fused)",
+    how = ("two launches per call: V^T x with a permuted copy of x, then the weight stream"
+           if path == "ring" else "one launch per call: W0 x, V^T x and the epilogue fused")
+    return {"kernel": f"{kernel} ({how})",
             "call": label, "path": path,
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
