@@ -11,10 +11,16 @@
 //               stages, completion on mbarriers (no multicast).
 //   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
 //               (128 x BN x 16, bf16 in, fp32 accumulate): the K loop over W0
-//               into accumulator A (columns 0..BN-1), then the r/64 low-rank
-//               blocks into accumulator B (columns 256..256+BN-1).  Each stage
-//               is released with tcgen05.commit; the finished tile is signalled
-//               to the epilogue the same way.
+//               into accumulator A, then the r/64 low-rank blocks into
+//               accumulator B.  With BN = 256 the two fill TMEM (A at column
+//               0, B at 256) and the next tile's MMAs wait for the epilogue;
+//               narrower tiles (and the swap mode) keep two sets of [A | B]
+//               (columns 0 and 256) and alternate, so the next tile's MMAs
+//               run while the epilogue drains the last.  (256-column tiles
+//               stay the faster choice for prefill: 1116 TFLOP/s single-set
+//               against 815 with 128-column double-set tiles on the Gemma-4
+//               gate/up call.)  Each stage is released with tcgen05.commit;
+//               the finished tile is signalled to the epilogue the same way.
 //   warps 2-5   epilogue: tcgen05.ld of both accumulators (one TMEM lane = one
 //               token row per thread), y = s * A + B in fp32, one rounding to
 //               bf16, stores with edge checks.
@@ -103,9 +109,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const uint32_t stages = (uint32_t)p.stages, stage_bytes = (uint32_t)p.stage_bytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(base + stages * stage_bytes);
     uint64_t *empty = full + stages;
-    uint64_t *tmem_full = empty + stages;
-    uint64_t *tmem_empty = tmem_full + 1;
-    uint64_t *drain = tmem_empty + 1;
+    uint64_t *tmem_full = empty + stages;  // [2]
+    uint64_t *tmem_empty = tmem_full + 2;  // [2]
+    uint64_t *drain = tmem_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *last_flag = abort_flag + 1;  // swap mode: this CTA adds up the tile's K ranges
@@ -117,14 +123,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const uint32_t b_rows = p.swap ? (uint32_t)p.mp : (uint32_t)p.BN;
     const uint32_t b_bytes = b_rows * kGemmBK * 2;
     const int units = p.num_tiles * p.ksplit;
+    // TMEM accumulators.  Tiles of at most 128 columns (and the swap mode's
+    // token tiles) use two sets, [A | B] at columns 0 and 256, so the MMAs of
+    // the next tile run while the epilogue drains this one; 256-column tiles
+    // use one set (A at 0, B at 256) and the MMAs wait for the drain.
+    const bool dbuf = p.swap || p.BN <= 128;
+    const uint32_t acc_b = dbuf ? 128u : kAccBCol;  // B's offset inside a set
+    auto acc_set = [&](uint32_t tc) -> uint32_t { return dbuf ? (tc & 1u) : 0u; };
+    auto acc_phase = [&](uint32_t tc) -> uint32_t { return dbuf ? (tc >> 1) & 1u : tc & 1u; };
 
     if (threadIdx.x == 0) {
         for (uint32_t i = 0; i < stages; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
-        mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tmem_full[i], 1);
+            mbar_init(&tmem_empty[i], 4);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -215,7 +231,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             const int kb0 = split * p.kb_split;
             const int nmain = min(nkb, kb0 + p.kb_split) - kb0;
             const int total = nmain + (split == 0 ? sg.lr_blocks : 0);
-            if (!warp_wait(tmem_empty, (tcount & 1u) ^ 1u, p, abort_flag)) {
+            const uint32_t set = acc_set(tcount);
+            if (!warp_wait(&tmem_empty[set], acc_phase(tcount) ^ 1u, p, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -232,7 +249,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     const uint64_t adesc = sw128_kmajor_desc(a_addr);
                     const uint64_t bdesc = sw128_kmajor_desc(b_addr);
                     const bool lowrank = i >= nmain;
-                    const uint32_t d = tmem_base + (lowrank ? kAccBCol : 0u);
+                    const uint32_t d = tmem_base + set * 256u + (lowrank ? acc_b : 0u);
                     const bool first = (i == 0) || (i == nmain);
 #pragma unroll
                     for (int k = 0; k < kGemmBK / 16; ++k) {
@@ -249,7 +266,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 }
             }
             if (!ok) break;
-            if (lane == 0) tc_commit(tmem_full);
+            if (lane == 0) tc_commit(&tmem_full[set]);
             __syncwarp();
             ++tcount;
         }
@@ -268,16 +285,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
             const TileInfo ti = tile_info(p, t);
             const GemmSeg &sg = p.seg[ti.seg];
-            if (!warp_wait(tmem_full, tcount & 1u, p, abort_flag)) break;
+            const uint32_t set = acc_set(tcount);
+            if (!warp_wait(&tmem_full[set], acc_phase(tcount), p, abort_flag)) break;
             tc_fence_after();
+            const uint32_t acc_addr = lane_addr + set * 256u;
             const int m = ti.m0 + row_in_tile;
             const bool lr = sg.lr_blocks > 0;
             const bool vec = ((reinterpret_cast<uintptr_t>(sg.y) & 15u) == 0) && (sg.ldy % 8 == 0);
             __nv_bfloat16 *yrow = sg.y + (size_t)m * sg.ldy;
             for (int c = 0; c < p.BN; c += 32) {
                 uint32_t a[32], b[32];
-                tmem_ld32(lane_addr + (uint32_t)c, a);
-                if (lr) tmem_ld32(lane_addr + kAccBCol + (uint32_t)c, b);
+                tmem_ld32(acc_addr + (uint32_t)c, a);
+                if (lr) tmem_ld32(acc_addr + acc_b + (uint32_t)c, b);
                 tmem_ld_wait();
                 const int nb = ti.n0 + c;
                 if (m < p.M && nb < sg.N) {
@@ -309,7 +328,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tmem_empty);
+            if (lane == 0) mbar_arrive(&tmem_empty[set]);
             ++tcount;
         }
     } else {
@@ -330,7 +349,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             const int tile = u / p.ksplit, split = u - tile * p.ksplit;
             const TileInfo ti = tile_info(p, tile);
             const GemmSeg &sg = p.seg[ti.seg];
-            bool ok = warp_wait(tmem_full, tcount & 1u, p, abort_flag);
+            const uint32_t set = acc_set(tcount);
+            bool ok = warp_wait(&tmem_full[set], acc_phase(tcount), p, abort_flag);
             if (p.ksplit > 1) {
                 uint32_t any_fail;
                 asm volatile(
@@ -353,8 +373,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             float *dp = p.part + ((size_t)p.ksplit * p.num_tiles + tile) * tile_stride + row_in_tile;
             for (int c = 0; c < mp; c += 32) {
                 uint32_t a[32], b[32];
-                tmem_ld32(lane_addr + (uint32_t)c, a);
-                if (lr_here) tmem_ld32(lane_addr + kAccBCol + (uint32_t)c, b);
+                tmem_ld32(lane_addr + set * 256u + (uint32_t)c, a);
+                if (lr_here) tmem_ld32(lane_addr + set * 256u + acc_b + (uint32_t)c, b);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -371,10 +391,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                     }
                 }
             }
-            // TMEM is read: the MMA warp may start the next unit.
+            // TMEM is read: the MMA warp may reuse this set.
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tmem_empty);
+            if (lane == 0) mbar_arrive(&tmem_empty[set]);
             ++tcount;
             if (p.ksplit == 1) continue;
             __threadfence();
@@ -436,7 +456,7 @@ void set_gemm_stages(GemmParams &p) {
 }
 
 size_t gemm_smem_bytes(const GemmParams &p) {
-    return 1024 + (size_t)p.stages * p.stage_bytes + (2 * kGemmMaxStages + 3) * 8 + 16;
+    return 1024 + (size_t)p.stages * p.stage_bytes + (2 * kGemmMaxStages + 5) * 8 + 16;
 }
 
 cudaError_t launch_gemm(const GemmParams &p, int num_sms, cudaStream_t stream) {
