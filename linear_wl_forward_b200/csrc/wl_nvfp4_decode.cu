@@ -74,7 +74,6 @@ constexpr int kRingThreads = FTH + 32;  // + the producer warp
 constexpr int kIssueLanes = 4;          // producer lanes issuing copies
 constexpr uint32_t kCodeBytes = 16 * 64 * kFp4StageKG;   // 16 KB: 16 rows x 1024 bytes
 constexpr uint32_t kScaleBytes = 16 * 8 * kFp4StageKG;   // 2 KB: 16 rows x 128 bytes
-constexpr int kKgPerWarp = kFp4StageKG / FW;              // k-groups of a stage per warp
 constexpr uint32_t kTOff = 8192;  // U unit: T (M x r fp32) after U (16 x 2r bytes <= 8 KB)
 constexpr uint32_t kRingSmemMax = 227 * 1024;
 constexpr int kFp4RingMaxBlocksPerSm = 4;
@@ -541,13 +540,17 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
     const int G = gridDim.x, c = blockIdx.x;
     const long long utot = P.utot;
     const long long u0 = range_start(utot, G, c), u1 = range_start(utot, G, c + 1);
-    // k-units: 128-column k-groups of NVFP4 codes, or 32-column groups of
-    // bf16 weights; a stage holds kFp4StageKG of them (1 KB of each row)
+    // k-units: 128-column k-groups of NVFP4 codes (16 per stage: 1 KB of
+    // each row, one TMA box), or 32-column groups of bf16 weights (32 per
+    // stage: 2 KB of each row, two boxes)
+    constexpr int KU = BF16 ? 2 * kFp4StageKG : kFp4StageKG;
+    constexpr uint32_t WB = 16u * 64u * KU;            // weight bytes of a stage
+    constexpr int NBOX = (int)(WB / kCodeBytes);       // 16-row x 1 KB boxes per stage
     constexpr uint32_t SCB = BF16 ? 0u : kScaleBytes;  // block scales of a stage
     const int K = P.K, M = P.M, Mp = P.Mp, nst = P.nst;
     const int nkg = BF16 ? (K + 31) / 32 : K / FKG;
     const uint32_t xstage = (BF16 ? 64u : 256u) * (uint32_t)Mp;  // bytes of permuted x per k-unit
-    const uint32_t sv_off = kCodeBytes + SCB + (uint32_t)kFp4StageKG * xstage;  // 16 row scales
+    const uint32_t sv_off = WB + SCB + (uint32_t)KU * xstage;     // 16 row scales
 
     if (warp == FW && lane < P.nseg) {
         // the tensor maps into the descriptor cache before the first copy
@@ -584,9 +587,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
             // (U unit) this projection's T, one row per token
             auto issue_dep = [&](int sl, const UnitCursor &c) {
                 if (c.st < nst) {
-                    const int kgs = min(kFp4StageKG, nkg - kFp4StageKG * c.st);
-                    bulk_load(ring + (size_t)sl * SB + kCodeBytes + SCB,
-                              reinterpret_cast<const uint8_t *>(P.xq) + (size_t)kFp4StageKG * c.st * xstage,
+                    const int kgs = min(KU, nkg - KU * c.st);
+                    bulk_load(ring + (size_t)sl * SB + WB + SCB,
+                              reinterpret_cast<const uint8_t *>(P.xq) + (size_t)KU * c.st * xstage,
                               (uint32_t)kgs * xstage, &full[sl]);
                 } else {
                     const Fp4Seg &S2 = P.seg[c.sp];
@@ -621,9 +624,12 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
                 const bool first = i == 0 || cu.st == 0;
                 const uint32_t sbytes = first ? 64u : 0u;
                 if (cu.st < nst) {
-                    const int kgs = min(kFp4StageKG, nkg - kFp4StageKG * cu.st);
-                    mbar_arrive_expect_tx(&full[slot], kCodeBytes + SCB + (uint32_t)kgs * xstage + sbytes);
-                    tma_2d(sb, &P.tm_c[cu.sp], (int)(kCodeBytes / 64) * cu.st, row0, &full[slot], pol);
+                    const int kgs = min(KU, nkg - KU * cu.st);
+                    mbar_arrive_expect_tx(&full[slot], WB + SCB + (uint32_t)kgs * xstage + sbytes);
+#pragma unroll
+                    for (int bx = 0; bx < NBOX; ++bx)
+                        tma_2d(sb + (size_t)bx * kCodeBytes, &P.tm_c[cu.sp], (int)(kCodeBytes / 64) * (NBOX * cu.st + bx),
+                               row0, &full[slot], pol);
                     if (!BF16)
                         tma_2d(sb + kCodeBytes, &P.tm_s[cu.sp], (int)(kScaleBytes / 64) * cu.st, row0, &full[slot], pol);
                 } else {
@@ -676,16 +682,17 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
                     // k-groups warp and warp + 8 of the stage; codes: row g at
                     // 1024 g; scales: row g at 128 g
 #pragma unroll
-                    for (int j = 0; j < kKgPerWarp; ++j) {
+                    for (int j = 0; j < KU / FW; ++j) {
                         const int kgl = warp + FW * j;
-                        if (kFp4StageKG * cu.st + kgl >= nkg) break;
-                        const uint32_t cb = sa + 64u * kgl + 16u * q;
+                        if (KU * cu.st + kgl >= nkg) break;
+                        // box kgl / 16, rows 1 KB apart inside it
+                        const uint32_t cb = sa + (uint32_t)(kgl >> 4) * kCodeBytes + 64u * (kgl & 15) + 16u * q;
                         if (BF16) {
                             // 32 columns of rows g and g + 8: the lane's eight
                             // (8q .. 8q + 7) are the logical columns 2q, 2q + 1,
                             // 2q + 8, 2q + 9 of two MMAs, as in x's copy
                             const uint4 w0 = lds128(cb + g * (kCodeBytes / 16)), w1 = lds128(cb + (g + 8) * (kCodeBytes / 16));
-                            const uint4 bx = xv ? lds128(sa + kCodeBytes + (uint32_t)(((kgl * Mp + g) * 4 + q) * 16))
+                            const uint4 bx = xv ? lds128(sa + WB + (uint32_t)(((kgl * Mp + g) * 4 + q) * 16))
                                                 : make_uint4(0u, 0u, 0u, 0u);
                             const uint32_t a1[4] = {w0.x, w1.x, w0.y, w1.y};
                             const uint32_t a2[4] = {w0.z, w1.z, w0.w, w1.w};
@@ -858,7 +865,8 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     p.ring = ring ? 1 : 0;
     if (!ring) return p.bf16 ? WL_ERR_UNSUPPORTED : WL_OK;
     const int nkg = p.bf16 ? (K + 31) / 32 : K / FKG;  // k-units
-    p.nst = (nkg + kFp4StageKG - 1) / kFp4StageKG;
+    const int ku = p.bf16 ? 2 * kFp4StageKG : kFp4StageKG;  // per stage (the kernel's KU)
+    p.nst = (nkg + ku - 1) / ku;
     long long ub = 0;
     for (int i = 0; i < p.nseg; ++i) {
         Fp4Seg &sg = p.seg[i];
@@ -868,9 +876,9 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     }
     p.utot = ub;
     p.grid = (int)std::min<long long>(num_sms, ub);
-    const uint32_t slot =
-        (kCodeBytes + (p.bf16 ? 0u : kScaleBytes) + (uint32_t)kFp4StageKG * (p.bf16 ? 64u : 256u) * p.Mp + 64u + 1023u) &
-        ~1023u;
+    const uint32_t slot = (16u * 64u * ku + (p.bf16 ? 0u : kScaleBytes) + (uint32_t)ku * (p.bf16 ? 64u : 256u) * p.Mp +
+                           64u + 1023u) &
+                          ~1023u;
     p.slot_bytes = (int)slot;
     const uint32_t fixed = 2u * FW * 32 * 2 * 16 + 32 + 1024;  // reduction buffers, flags, alignment
     int ns = (int)((kRingSmemMax - fixed) / (slot + 16));
