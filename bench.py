@@ -152,7 +152,7 @@ def call_path(M, projs_nr, K=None):
     import linear_wl_forward_b200 as wl
 
     rows = sum(n for n, _ in projs_nr)
-    if (K is not None and M <= 8 and 2 * rows * K >= (64 << 20) and not (M >= 5 and rows >= 32768)
+    if (K is not None and M <= 8 and 2 * rows * K >= (64 << 20)
             and all(r % 8 == 0 and r <= 256 for _, r in projs_nr)):
         return "ring"
     if M <= 4 or (M <= wl.DECODE_MAX_M and rows < 8192):
@@ -335,7 +335,8 @@ def decode_roofline(wl, peaks, call="gemma3_gate_up", seconds=1.0):
     ms = st["median_ms"]
     achieved = call_bytes / (ms * 1e-3) / 1e9
     path = call_path(M, [(N, r) for N in Ns], K)
-    kernel = {"rows": "rows_kernel", "decode": "decode_kernel", "ring": "ring_kernel<true>"}.get(path, "gemm_kernel")
+    ring = f"ring_kernel<true, {48 if M <= 2 else 32}>"  # bf16 rows of 3 or 2 KB per stage
+    kernel = {"rows": "rows_kernel", "decode": "decode_kernel", "ring": ring}.get(path, "gemm_kernel")
     traffic = traffic_from_profile(kernel, call)
     how = ("two launches per call: V^T x with a permuted copy of x, then the weight stream"
            if path == "ring" else "one launch per call: W0 x, V^T x and the epilogue fused")

@@ -87,8 +87,8 @@ typedef struct {
 } wl_proj;
 
 /* Which kernels a forward call uses.  WL_PATH_AUTO takes the persistent ring
- * for calls of at most 8 tokens whose weights total at least 64 MB (except
- * 5-8 tokens over 32768 or more output rows) when the call fits it; else a
+ * for calls of at most 8 tokens whose weights total at least 64 MB when the
+ * call fits it; else a
  * decode kernel for M <= 4, and for M <= WL_DECODE_MAX_M when the call's
  * projections total fewer than 8192 output rows; otherwise the tensor-core
  * GEMM.  Of the two decode

@@ -248,16 +248,14 @@ wl_status build_prefetch(const wl_range *ranges, int n, PrefetchList &pf) {
 //   q/k/v 1536 x 1152, M = 8: decode 19.5 us, GEMM 22.9 us
 // Large calls of at most 8 tokens take the persistent ring: at least 64 MB
 // of bf16 weights (the Gemma-4-31B projections; measured against the other
-// kernels: q/k/v 57 against 66 us at M = 1, down 68 against 129 us at M = 2,
-// o 56 against 145 us at M = 8), except wide calls of 5-8 tokens over 32768 or
-// more rows, where the tensor-core GEMM is faster (gate/up 136 against 155 us
-// at M = 8).
+// kernels, us at M = 1 / 8: gate/up 88.7 / 126.6 against 122.5 (decode) /
+// 133.7 (GEMM), down 50.8 / 76.7 against 72.0 / 106.2, q/k/v 45.9 against
+// 66.3 at M = 1).
 bool auto_ring(int M, int K, const wl_proj *projs, int P) {
     if (M > kFp4MaxM) return false;
     long long rows = 0;
     for (int i = 0; i < P; ++i) rows += projs[i].N;
-    if (2LL * rows * K < (64LL << 20)) return false;
-    return !(M >= 5 && rows >= 32768);
+    return 2LL * rows * K >= (64LL << 20);
 }
 
 bool auto_decode(int M, const wl_proj *projs, int P) {

@@ -242,6 +242,7 @@ struct Fp4Params {
     int bf16;             // 1: W0 in bf16 (codes = the bf16 rows, no scales, tensor scale 1); ring stream only
     int ring;             // 1: ring stream, 0: block stream
     int grid, ns, slot_bytes, smem, nst;
+    int ku;               // k-units per stage (128-column groups for NVFP4, 32-column for bf16)
     long long utot;
     float2 *parts;        // [grid][2][16 * kFp4MaxM] partial (z, d) of blocks split between CTAs
     unsigned int *bcnt;   // [total_blocks] CTAs done with a split block (zeroed, self-resetting)

@@ -71,7 +71,7 @@ constexpr int FTH = 32 * FW;
 constexpr int FKG = kFp4KGroup;   // 128 columns per k-group
 constexpr int kPrepThreads = 256;
 constexpr int kRingThreads = FTH + 32;  // + the producer warp
-constexpr int kIssueLanes = 4;          // producer lanes issuing copies
+constexpr int kIssueLanes = 2;          // producer lanes issuing copies
 constexpr uint32_t kCodeBytes = 16 * 64 * kFp4StageKG;   // 16 KB: 16 rows x 1024 bytes
 constexpr uint32_t kScaleBytes = 16 * 8 * kFp4StageKG;   // 2 KB: 16 rows x 128 bytes
 constexpr uint32_t kTOff = 8192;  // U unit: T (M x r fp32) after U (16 x 2r bytes <= 8 KB)
@@ -523,7 +523,7 @@ __device__ __forceinline__ int cta_of(long long utot, int G, long long u) {
 
 }  // namespace
 
-template <bool BF16>
+template <bool BF16, int KU>
 __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_constant__ Fp4Params P) {
     pdl_launch_dependents();
     extern __shared__ uint8_t dyn_smem[];
@@ -540,10 +540,12 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
     const int G = gridDim.x, c = blockIdx.x;
     const long long utot = P.utot;
     const long long u0 = range_start(utot, G, c), u1 = range_start(utot, G, c + 1);
-    // k-units: 128-column k-groups of NVFP4 codes (16 per stage: 1 KB of
-    // each row, one TMA box), or 32-column groups of bf16 weights (32 per
-    // stage: 2 KB of each row, two boxes)
-    constexpr int KU = BF16 ? 2 * kFp4StageKG : kFp4StageKG;
+    // k-units: 128-column k-groups of NVFP4 codes (KU = 16 per stage: 1 KB
+    // of each row, one TMA box), or 32-column groups of bf16 weights (KU =
+    // 48 or 32 per stage: 3 or 2 KB of each row, as many boxes).  Long runs
+    // of each row per request stream faster (measured on the Gemma-4 gate/up
+    // call at M = 1: 1 KB 119.8 us, 2 KB 102.7, 3 KB 90.5, 4 KB 92.6).
+    static_assert(KU % FW == 0 && KU % kFp4StageKG == 0, "k-units of a stage");
     constexpr uint32_t WB = 16u * 64u * KU;            // weight bytes of a stage
     constexpr int NBOX = (int)(WB / kCodeBytes);       // 16-row x 1 KB boxes per stage
     constexpr uint32_t SCB = BF16 ? 0u : kScaleBytes;  // block scales of a stage
@@ -865,7 +867,11 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     p.ring = ring ? 1 : 0;
     if (!ring) return p.bf16 ? WL_ERR_UNSUPPORTED : WL_OK;
     const int nkg = p.bf16 ? (K + 31) / 32 : K / FKG;  // k-units
-    const int ku = p.bf16 ? 2 * kFp4StageKG : kFp4StageKG;  // per stage (the kernel's KU)
+    // per stage (the kernel's KU): bf16 rows of 3 KB per stage for up to two
+    // token rows of x, of 2 KB above (the x slices grow with the tokens and
+    // the ring must keep enough slots)
+    const int ku = p.bf16 ? (p.Mp <= 2 ? 3 * kFp4StageKG : 2 * kFp4StageKG) : kFp4StageKG;
+    p.ku = ku;
     p.nst = (nkg + ku - 1) / ku;
     long long ub = 0;
     for (int i = 0; i < p.nseg; ++i) {
@@ -923,16 +929,23 @@ cudaError_t launch_fp4(const Fp4Params &p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (p.ring) {
         if (!g_ring_attr.load(std::memory_order_acquire)) {
-            e = cudaFuncSetAttribute(ring_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+            e = cudaFuncSetAttribute(ring_kernel<false, kFp4StageKG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kRingSmemMax);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(ring_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+                e = cudaFuncSetAttribute(ring_kernel<true, 2 * kFp4StageKG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(ring_kernel<true, 3 * kFp4StageKG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
             if (e != cudaSuccess) return e;
             g_ring_attr.store(true, std::memory_order_release);
         }
         cfg.blockDim = dim3(kRingThreads);
         cfg.gridDim = dim3((unsigned)p.grid);
         cfg.dynamicSmemBytes = (size_t)p.smem;
-        return p.bf16 ? cudaLaunchKernelEx(&cfg, ring_kernel<true>, p) : cudaLaunchKernelEx(&cfg, ring_kernel<false>, p);
+        if (!p.bf16) return cudaLaunchKernelEx(&cfg, ring_kernel<false, kFp4StageKG>, p);
+        return p.ku == 3 * kFp4StageKG ? cudaLaunchKernelEx(&cfg, ring_kernel<true, 3 * kFp4StageKG>, p)
+                                       : cudaLaunchKernelEx(&cfg, ring_kernel<true, 2 * kFp4StageKG>, p);
     }
     cfg.blockDim = dim3(FTH);
     cfg.gridDim = dim3((unsigned)p.total_blocks);
