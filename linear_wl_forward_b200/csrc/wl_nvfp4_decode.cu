@@ -1,3 +1,10 @@
+// The two-launch decode kernels: a prep launch (V^T x and a permuted copy of
+// x) followed by a weight stream.  They serve the NVFP4 shared block (below)
+// and, through the persistent ring with bf16 weight tiles, the large bf16
+// calls of at most 8 tokens (WL_PATH_RING; the ring section at the end of this
+// comment).  The parameter block is shared (Fp4Params; bf16 = 1 for the bf16
+// ring, whose "codes" are the bf16 rows, with no scales and tensor scale 1).
+//
 // Decode with an NVFP4 shared block: y = s (.) (W0 x) + U (V^T x) where W0 is
 // stored as FP4 E2M1 codes (two per byte, element 2i in the low nibble of
 // byte i), one FP8 E4M3 scale per 16 consecutive elements of a row, and one
@@ -54,6 +61,15 @@
 // blocks (otherwise): one CTA per 16-row block, eight warps splitting the
 //   k-groups, four k-groups' loads in flight per warp straight into
 //   registers, then the U rows and T from global memory.
+//
+// bf16 ring (ring_kernel<true, KU>): the same persistent ring with stages of
+//   16 rows x KU 32-column groups of bf16 W0 (KU = 48 for up to two tokens,
+//   32 above: 3 or 2 KB of each row per stage, as many 16-row x 1 KB TMA
+//   boxes).  Longer runs of each row per request stream faster (Gemma-4
+//   gate/up, M = 1: 1 KB 119.8 us, 2 KB 102.7, 3 KB 88.7).  Lane q's eight
+//   consecutive columns of a 32-column group are the logical columns 2q,
+//   2q + 1, 2q + 8, 2q + 9 of two MMAs, and the prep launch writes x in the
+//   same order: [K/32][token][4][8] bf16.
 #include <cuda_fp16.h>
 
 #include <algorithm>
