@@ -89,11 +89,10 @@ constexpr int kPrepThreads = 256;
 constexpr int kRingThreads = FTH + 32;  // + the producer warp
 constexpr int kIssueLanes = 2;          // producer lanes issuing copies
 constexpr uint32_t kCodeBytes = 16 * 64 * kFp4StageKG;   // 16 KB: 16 rows x 1024 bytes
-constexpr uint32_t kScaleBytes = 16 * 8 * kFp4StageKG;   // 2 KB: 16 rows x 128 bytes
 constexpr uint32_t kTOff = 8192;  // U unit: T (M x r fp32) after U (16 x 2r bytes <= 8 KB)
 constexpr uint32_t kRingSmemMax = 227 * 1024;
-constexpr int kFp4RingMaxBlocksPerSm = 4;
-constexpr int kFp4RingMinK = 16384;
+constexpr int kFp4RingMinK = 8192;         // NVFP4 calls with K at least this take the ring
+constexpr int kFp4RingMinBlocks = 2048;    // ... and so do calls of at least this many 16-row blocks
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -564,7 +563,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
     static_assert(KU % FW == 0 && KU % kFp4StageKG == 0, "k-units of a stage");
     constexpr uint32_t WB = 16u * 64u * KU;            // weight bytes of a stage
     constexpr int NBOX = (int)(WB / kCodeBytes);       // 16-row x 1 KB boxes per stage
-    constexpr uint32_t SCB = BF16 ? 0u : kScaleBytes;  // block scales of a stage
+    constexpr uint32_t SCB = BF16 ? 0u : 16u * 8u * KU;  // block scales of a stage (8 bytes per row and k-group)
     const int K = P.K, M = P.M, Mp = P.Mp, nst = P.nst;
     const int nkg = BF16 ? (K + 31) / 32 : K / FKG;
     const uint32_t xstage = (BF16 ? 64u : 256u) * (uint32_t)Mp;  // bytes of permuted x per k-unit
@@ -649,7 +648,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
                         tma_2d(sb + (size_t)bx * kCodeBytes, &P.tm_c[cu.sp], (int)(kCodeBytes / 64) * (NBOX * cu.st + bx),
                                row0, &full[slot], pol);
                     if (!BF16)
-                        tma_2d(sb + kCodeBytes, &P.tm_s[cu.sp], (int)(kScaleBytes / 64) * cu.st, row0, &full[slot], pol);
+                        tma_2d(sb + WB, &P.tm_s[cu.sp], 2 * KU * cu.st, row0, &full[slot], pol);
                 } else {
                     mbar_arrive_expect_tx(&full[slot], 32u * (uint32_t)S.r + 4u * (uint32_t)(M * S.r) + sbytes);
                     tma_2d(sb, &P.tm_u[cu.sp], 0, row0, &full[slot], pol);
@@ -719,10 +718,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) ring_kernel(const __grid_cons
                             continue;
                         }
                         const uint4 c0 = lds128(cb + g * (kCodeBytes / 16)), c1 = lds128(cb + (g + 8) * (kCodeBytes / 16));
-                        const uint32_t sbs = sa + kCodeBytes + 8u * kgl + 2u * q;
-                        const uint16_t s0 = lds16(sbs + g * (kScaleBytes / 16)), s1 = lds16(sbs + (g + 8) * (kScaleBytes / 16));
+                        const uint32_t sbs = sa + WB + 8u * kgl + 2u * q;
+                        const uint16_t s0 = lds16(sbs + g * (SCB / 16)), s1 = lds16(sbs + (g + 8) * (SCB / 16));
                         uint4 xf[4];
-                        const uint32_t xb = sa + kCodeBytes + SCB;
+                        const uint32_t xb = sa + WB + SCB;
 #pragma unroll
                         for (int t = 0; t < 4; ++t)
                             xf[t] = xv ? lds128(xb + (uint32_t)((((kgl * 4 + t) * Mp + g) * 4 + q) * 16))
@@ -874,19 +873,19 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     for (int i = 0; i < p.nseg; ++i)
         ring = ring && p.seg[i].r <= kFp4RingMaxRank && (reinterpret_cast<uintptr_t>(p.seg[i].s) & 15u) == 0 &&
                (p.bf16 || (reinterpret_cast<uintptr_t>(p.seg[i].scales) & 15u) == 0);
-    // NVFP4: and when the call has few row blocks per SM, each of a long K:
-    // the ring balances them evenly over the SMs.  Otherwise one CTA per
-    // block streams faster (measured on the Gemma-4-31B families: the ring
-    // wins only for down, 5376 x 21504; q 8192 x 5376 and o 5376 x 8192, also
-    // few blocks, run faster per block).  bf16 weights: the caller decides.
-    if (!p.bf16) ring = ring && p.total_blocks <= kFp4RingMaxBlocksPerSm * num_sms && K >= kFp4RingMinK;
+    // NVFP4: and when K is long or the call has many row blocks; otherwise
+    // one CTA per block streams faster (measured on the Gemma-4-31B families
+    // at M = 1, rank 256, ring against block stream: gate/up 69.7 / 72.0 us,
+    // down 35.6 / 41.0, o 5376 x 8192 24.3 / 26.2, but q 8192 x 5376 27.3 /
+    // 24.5).  bf16 weights: the caller decides.
+    if (!p.bf16) ring = ring && (K >= kFp4RingMinK || p.total_blocks >= kFp4RingMinBlocks);
     p.ring = ring ? 1 : 0;
     if (!ring) return p.bf16 ? WL_ERR_UNSUPPORTED : WL_OK;
     const int nkg = p.bf16 ? (K + 31) / 32 : K / FKG;  // k-units
     // per stage (the kernel's KU): bf16 rows of 3 KB per stage for up to two
     // token rows of x, of 2 KB above (the x slices grow with the tokens and
     // the ring must keep enough slots)
-    const int ku = p.bf16 ? (p.Mp <= 2 ? 3 * kFp4StageKG : 2 * kFp4StageKG) : kFp4StageKG;
+    const int ku = p.Mp <= 2 ? (p.bf16 ? 3 : 2) * kFp4StageKG : (p.bf16 ? 2 : 1) * kFp4StageKG;
     p.ku = ku;
     p.nst = (nkg + ku - 1) / ku;
     long long ub = 0;
@@ -898,7 +897,7 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
     }
     p.utot = ub;
     p.grid = (int)std::min<long long>(num_sms, ub);
-    const uint32_t slot = (16u * 64u * ku + (p.bf16 ? 0u : kScaleBytes) + (uint32_t)ku * (p.bf16 ? 64u : 256u) * p.Mp +
+    const uint32_t slot = (16u * 64u * ku + (p.bf16 ? 0u : 16u * 8u * ku) + (uint32_t)ku * (p.bf16 ? 64u : 256u) * p.Mp +
                            64u + 1023u) &
                           ~1023u;
     p.slot_bytes = (int)slot;
@@ -919,7 +918,7 @@ wl_status plan_fp4(Fp4Params &p, int num_sms, bool encode_maps) {
         if ((st = encode_map_2d_u32(&p.tm_c[i], sg.codes, wwords, sg.N, wwords * 4, kCodeBytes / 64, 16)) != WL_OK)
             return st;
         if (!p.bf16 &&
-            (st = encode_map_2d_u32(&p.tm_s[i], sg.scales, (uint64_t)K / 64, sg.N, (uint64_t)K / 16, kScaleBytes / 64, 16)) !=
+            (st = encode_map_2d_u32(&p.tm_s[i], sg.scales, (uint64_t)K / 64, sg.N, (uint64_t)K / 16, 2u * ku, 16)) !=
                 WL_OK)
             return st;
         if (sg.r > 0 &&
@@ -948,6 +947,9 @@ cudaError_t launch_fp4(const Fp4Params &p, cudaStream_t stream) {
             e = cudaFuncSetAttribute(ring_kernel<false, kFp4StageKG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kRingSmemMax);
             if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(ring_kernel<false, 2 * kFp4StageKG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
+            if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(ring_kernel<true, 2 * kFp4StageKG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRingSmemMax);
             if (e == cudaSuccess)
@@ -959,7 +961,9 @@ cudaError_t launch_fp4(const Fp4Params &p, cudaStream_t stream) {
         cfg.blockDim = dim3(kRingThreads);
         cfg.gridDim = dim3((unsigned)p.grid);
         cfg.dynamicSmemBytes = (size_t)p.smem;
-        if (!p.bf16) return cudaLaunchKernelEx(&cfg, ring_kernel<false, kFp4StageKG>, p);
+        if (!p.bf16)
+            return p.ku == 2 * kFp4StageKG ? cudaLaunchKernelEx(&cfg, ring_kernel<false, 2 * kFp4StageKG>, p)
+                                           : cudaLaunchKernelEx(&cfg, ring_kernel<false, kFp4StageKG>, p);
         return p.ku == 3 * kFp4StageKG ? cudaLaunchKernelEx(&cfg, ring_kernel<true, 3 * kFp4StageKG>, p)
                                        : cudaLaunchKernelEx(&cfg, ring_kernel<true, 2 * kFp4StageKG>, p);
     }

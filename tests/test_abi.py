@@ -144,23 +144,25 @@ def test_nvfp4_validation(L):
 
 
 def test_nvfp4_plan_picks_the_stream():
-    """wl_describe_nvfp4_plan: the ring stream for K % 256 == 0, K >= 16384,
-    ranks <= 256, 16-byte-aligned scales and at most 4 row blocks per SM; one
-    CTA per 16-row block otherwise.  The ring's shared memory fits a CTA and its
+    """wl_describe_nvfp4_plan: the ring stream for K % 256 == 0, ranks <= 256,
+    16-byte-aligned scales and K >= 8192 or at least 2048 row blocks; one CTA
+    per 16-row block otherwise.  The ring's shared memory fits a CTA and its
     units cover the call."""
     ring = wl.describe_nvfp4_plan(1, 21504, [(5376, 256)])      # Gemma-4 down
     assert ring["ring"] == 1 and ring["grid"] == 148
-    assert ring["units"] == 336 * (11 + 1)           # 336 blocks x (11 stages of 2048 columns + U) each
-    assert ring["smem_bytes"] <= 227 * 1024 and ring["stages"] >= 4
+    assert ring["units"] == 336 * (6 + 1)            # 336 blocks x (6 stages of 4096 columns + U) each
+    assert ring["smem_bytes"] <= 227 * 1024 and ring["stages"] >= 2
     assert ring["prep_grid"] == ring["prep_slices"]
     assert ring["prep_slices"] * ring["prep_rows"] >= 21504
     gate_up = wl.describe_nvfp4_plan(1, 5376, [(21504, 256), (21504, 256)])
-    assert gate_up["ring"] == 0 and gate_up["grid"] == 2 * 1344   # 2688 blocks > 4 per SM
+    assert gate_up["ring"] == 1 and gate_up["grid"] == 148           # 2688 blocks
     assert gate_up["prep_grid"] == 2 * gate_up["prep_slices"]
-    assert wl.describe_nvfp4_plan(1, 8192, [(5376, 256)])["ring"] == 0       # Gemma-4 o: K < 16384
+    q = wl.describe_nvfp4_plan(1, 5376, [(8192, 256)])
+    assert q["ring"] == 0 and q["grid"] == 8192 // 16                 # 512 blocks over a short K
+    assert wl.describe_nvfp4_plan(1, 8192, [(5376, 256)])["ring"] == 1       # Gemma-4 o: K = 8192
     for M in range(1, wl.NVFP4_MAX_M + 1):
         p = wl.describe_nvfp4_plan(M, 16384, [(700, 256)])
-        assert p["ring"] == 1 and p["smem_bytes"] <= 227 * 1024 and p["stages"] >= 4
+        assert p["ring"] == 1 and p["smem_bytes"] <= 227 * 1024 and p["stages"] >= 2
     assert wl.describe_nvfp4_plan(1, 1152, [(300, 16)])["ring"] == 0          # K % 256 != 0
     assert wl.describe_nvfp4_plan(1, 16384, [(300, 512)])["ring"] == 0        # rank > 256
     assert wl.describe_nvfp4_plan(1, 16384, [(300, 16, 2)])["ring"] == 0      # scales at +2 bytes
@@ -168,4 +170,4 @@ def test_nvfp4_plan_picks_the_stream():
     blocks = wl.describe_nvfp4_plan(1, 1152, [(300, 16)])
     assert blocks["grid"] == (300 + 15) // 16
     tiny = wl.describe_nvfp4_plan(1, 16384, [(16, 24)])
-    assert tiny["ring"] == 1 and tiny["grid"] == tiny["units"] == 8 + 1
+    assert tiny["ring"] == 1 and tiny["grid"] == tiny["units"] == 4 + 1   # 4 stages of 4096 columns + U

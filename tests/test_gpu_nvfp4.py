@@ -83,10 +83,11 @@ def test_nvfp4_ring_stacked_split_blocks(M):
 
 
 def test_nvfp4_ring_one_block_over_many_ctas():
-    """16 rows, K = 21504: one block of 11 stages and a U unit, one unit per
-    CTA, so 12 CTAs each hold a part of the same block."""
+    """16 rows, K = 21504: one block of 6 stages (4096 columns, the last one
+    ragged) and a U unit, one unit per CTA, so 7 CTAs each hold a part of the
+    same block."""
     x, host, projs = _case(41, 1, [16], 21504, [256])
-    assert wl.describe_nvfp4_plan(1, 21504, [(16, 256)])["grid"] == 12
+    assert wl.describe_nvfp4_plan(1, 21504, [(16, 256)])["grid"] == 7
     _check(x, host, projs, ring=1)
 
 
