@@ -103,9 +103,10 @@ typedef enum {
     WL_PATH_ROWS = 3,   /* row-stream decode kernel (register-fed warp MMA, K split over CTA
                            clusters) for short calls; WL_ERR_UNSUPPORTED for calls it does not fit */
     WL_PATH_RING = 4    /* persistent ring decode (a V^T x launch, then one CTA per SM streaming
-                           16-row x 512-column weight tiles by TMA, the call's work split evenly
-                           over the SMs) for 1 <= M <= 8, ranks <= 256 and multiples of 8, U, V
-                           and s 16-byte aligned; WL_ERR_UNSUPPORTED otherwise */
+                           16-row x 1536-column (M <= 2) or x 1024-column weight tiles by TMA,
+                           the call's work split evenly over the SMs) for 1 <= M <= 8, ranks
+                           <= 256 and multiples of 8, U, V and s 16-byte aligned;
+                           WL_ERR_UNSUPPORTED otherwise */
 } wl_path;
 
 #define WL_DECODE_MAX_M 16
